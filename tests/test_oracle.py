@@ -1,0 +1,274 @@
+"""Pins for the float64 oracle: it is checked against things other than itself.
+
+Each test states what it pins and which plausible slip it would catch.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+from oracle import dsa_ref as R
+from long_context_sparse_04_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------
+# P8: number formats against an independent decoder (torch casts)
+# --------------------------------------------------------------------------
+
+def test_e4m3_decoder_matches_torch_on_all_codes():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = R.e4m3_decode(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert nan.sum() == 2                      # 0x7F and 0xFF only
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x80] == 0.0
+
+
+def test_bf16_decoder_matches_torch():
+    import torch
+    bits = np.random.default_rng(0).integers(0, 2 ** 16, size=5000).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]     # drop inf/nan patterns
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(ref, R.bf16_decode(bits))
+
+
+# --------------------------------------------------------------------------
+# P1: brute force, pure Python loops, L <= 64
+# --------------------------------------------------------------------------
+
+def _brute_indexer(q8, qs, w, k8, ks, klen):
+    """Scalar loops over the definition, decoding each byte on its own."""
+    def dec(c):                                  # OCP e4m3, written again by hand
+        s = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 15, c & 7
+        return s * (2.0 ** -6) * m / 8 if e == 0 else s * 2.0 ** (e - 7) * (1 + m / 8)
+    out = []
+    for s_ in range(klen):
+        acc = 0.0
+        for j in range(len(w)):
+            dot = 0.0
+            for d in range(len(k8[s_])):
+                dot += dec(int(q8[j][d])) * float(qs[j]) * dec(int(k8[s_][d])) * float(ks[s_])
+            acc += float(w[j]) * (dot if dot > 0 else 0.0)
+        out.append(acc)
+    return out
+
+
+def test_indexer_brute_force_fp8():
+    cfg = I.CONFIGS["prefill_8k"].replace(seq_len=48, h_idx=3, d_idx=16, topk=8,
+                                         n_heads=2, d_c=8, d_r=4, plant_frac=0.1)
+    inp = I.generate(cfg, threads=1)
+    for t in (0, 5, 31, 47):
+        got = R.row_scores(inp, t)
+        ref = _brute_indexer(inp["q_idx"][t], inp["q_scale"][t], inp["w"][t],
+                             inp["k_idx"], inp["k_scale"], t + 1)
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_mla_brute_force():
+    rng = np.random.default_rng(1)
+    H, dc, dr, n = 3, 6, 2, 9
+    q = rng.standard_normal((H, dc + dr))
+    kv = rng.standard_normal((n, dc + dr))
+    scale = 0.37
+    o, lse = R.sparse_mla_row(q, kv, dc, scale)
+    for i in range(H):
+        z = [scale * sum(q[i][d] * kv[s][d] for d in range(dc + dr)) for s in range(n)]
+        den = sum(math.exp(v) for v in z)
+        assert abs(lse[i] - math.log(den)) < 1e-12
+        for d in range(dc):
+            ref = sum(math.exp(z[s]) / den * kv[s][d] for s in range(n))
+            assert abs(o[i][d] - ref) < 1e-12
+
+
+def test_lse_matches_library_logsumexp():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((4, 10)) * 3
+    kv = rng.standard_normal((50, 10))
+    _, lse = R.sparse_mla_row(q, kv, 7, 0.9)
+    np.testing.assert_allclose(lse, scipy.special.logsumexp(0.9 * q @ kv.T, axis=1), rtol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# P2: top-k equals a full stable sort, with ties and signed zeros
+# --------------------------------------------------------------------------
+
+def _brute_topk(scores, k):
+    order = sorted(range(len(scores)), key=lambda s: (-float(scores[s]), s))[:k]
+    order = sorted(order)
+    return order + [-1] * (k - len(order))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_equals_stable_sort(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(0, 40))
+    vals = rng.choice([-1.5, -0.0, 0.0, 0.25, 0.25, 1.0, 2.0, 3.5], size=n) \
+        if seed % 2 else rng.standard_normal(n).round(1)
+    for k in (1, 3, 7, 40, 64):
+        assert list(R.topk_row(vals, k)) == _brute_topk(vals, k)
+
+
+def test_topk_signed_zero_and_degenerate():
+    v = np.array([0.0, -0.0, 0.0, -0.0, -1.0])
+    assert list(R.topk_row(v, 2)) == [0, 1]          # -0 == +0: lower index wins
+    assert list(R.topk_row(np.zeros(0), 4)) == [-1, -1, -1, -1]
+    assert list(R.topk_row(np.array([5.0, 1.0]), 4)) == [0, 1, -1, -1]
+    assert R.kth_score(np.array([3.0, 9.0, 1.0, 7.0]), 2) == 7.0
+    assert R.kth_score(np.array([3.0, 9.0]), 5) == 3.0
+
+
+# --------------------------------------------------------------------------
+# P3: k >= visible keys makes sparse MLA the dense MLA
+# --------------------------------------------------------------------------
+
+def test_full_k_equals_dense_attention():
+    inp = I.generate(I.CONFIGS["tiny_fp32"].replace(seq_len=40), threads=1)
+    res = R.dsa_forward_rows(inp, range(40), topk=64)
+    lat = inp["latent"].astype(np.float64)
+    for t, idx, o, lse in zip(res["rows"], res["idx"], res["out"], res["lse"]):
+        assert list(idx[: t + 1]) == list(range(t + 1)) and (idx[t + 1:] == -1).all()
+        z = inp["sm_scale"] * inp["q"][t].astype(np.float64) @ lat[: t + 1].T
+        p = scipy.special.softmax(z, axis=1)
+        np.testing.assert_allclose(o, p @ lat[: t + 1, :64], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse, scipy.special.logsumexp(z, axis=1), rtol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# P4: outputs are convex combinations of the selected value latents
+# --------------------------------------------------------------------------
+
+def test_output_is_convex_combination():
+    inp = I.generate(I.CONFIGS["tiny_fp32"], threads=1)
+    res = R.dsa_forward_rows(inp, [3, 100, 255])
+    lat = inp["latent"].astype(np.float64)
+    for t, idx, o, lse in zip(res["rows"], res["idx"], res["out"], res["lse"]):
+        sel = idx[idx >= 0]
+        assert len(sel) == min(64, t + 1)
+        c = lat[sel, :64]
+        assert (o >= c.min(axis=0) - 1e-12).all() and (o <= c.max(axis=0) + 1e-12).all()
+        z = inp["sm_scale"] * inp["q"][t].astype(np.float64) @ lat[sel].T
+        np.testing.assert_allclose(np.exp(z - lse[:, None]).sum(axis=1), 1.0, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# P5: the page's single-head ReLU(q.k/sqrt(d_I)) is the H_I=1 special case
+# --------------------------------------------------------------------------
+
+def test_single_head_reduction():
+    rng = np.random.default_rng(3)
+    for d in (32, 64, 128):
+        q = rng.standard_normal(d)
+        k = rng.standard_normal((100, d))
+        np.testing.assert_allclose(R.indexer_row(q[None], np.array([1 / math.sqrt(d)]), k),
+                                   R.indexer_row_single_head(q, k), rtol=1e-13, atol=1e-15)
+
+
+def test_indexer_weights_and_heads_not_transposed():
+    # distinct per-head weights: a swapped (t, j) index or a dropped head changes I
+    q = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]])
+    w = np.array([2.0, -3.0, 0.5])
+    k = np.array([[1.0, 2.0], [-1.0, 1.0], [-1.0, -1.0]])
+    # hand evaluation: s0 dots (1,2,3) -> 2-6+1.5; s1 (-1,1,0) -> -3; s2 all <= 0 -> 0
+    np.testing.assert_allclose(R.indexer_row(q, w, k), [-2.5, -3.0, 0.0])
+
+
+# --------------------------------------------------------------------------
+# P6: absorbed MLA equals MLA with explicit W_UK / W_UV up-projections
+# --------------------------------------------------------------------------
+
+def test_absorbed_equals_unabsorbed():
+    rng = np.random.default_rng(4)
+    H, d_h, d_v, d_c, d_r, n = 4, 12, 10, 16, 6, 30
+    c = rng.standard_normal((n, d_c))
+    kr = rng.standard_normal((n, d_r))
+    qn = rng.standard_normal((H, d_h))
+    qr = rng.standard_normal((H, d_r))
+    w_uk = rng.standard_normal((H, d_h, d_c)) / 3
+    w_uv = rng.standard_normal((H, d_v, d_c)) / 3
+    u_ref = R.unabsorbed_mla_row(qn, qr, c, kr, w_uk, w_uv)
+    q_abs = np.concatenate([np.einsum("hdc,hd->hc", w_uk, qn), qr], axis=1)
+    o, _ = R.sparse_mla_row(q_abs, np.concatenate([c, kr], axis=1), d_c, 1 / math.sqrt(d_h + d_r))
+    u = np.einsum("hvc,hc->hv", w_uv, o)
+    np.testing.assert_allclose(u, u_ref, rtol=1e-11, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# P7: counts the pages print
+# --------------------------------------------------------------------------
+
+def test_page_counts():
+    g = json.load(open(os.path.join(GOLDEN, "page_counts.json")))
+    e = g["causal_pairs_131072"]
+    cfg = I.CONFIGS["prefill_64k"].replace(seq_len=e["L"])
+    _, klen = I.row_layout(cfg)
+    pairs = int(klen.astype(np.int64).sum())
+    assert pairs == 8_590_000_128
+    assert abs(pairs - e["value"]) <= e["rel_tol"] * e["value"]
+    s = g["sparsity_k2048_L131072"]
+    assert 1 - s["k"] / s["L"] > s["value"]
+    f = g["fraction_k2048_L128000"]
+    assert abs(f["k"] / f["L"] - f["value"]) <= f["rel_tol"] * f["value"]
+    assert I.CONFIGS["decode_128k_paged"].topk == g["topk_value"]["value"]
+
+
+# --------------------------------------------------------------------------
+# cache addressing: a paged layout and a contiguous layout of the same blocks
+# give the same results (block table indirection done right)
+# --------------------------------------------------------------------------
+
+def test_paged_equals_contiguous():
+    base = I.CONFIGS["decode_128k_paged"].replace(
+        ctx_lo=150, ctx_hi=300, n_seqs=3, h_idx=4, d_idx=16, topk=32, n_heads=2, d_c=8, d_r=4)
+    a = I.generate(base, threads=1)
+    b = I.generate(base.replace(paged=False), threads=1)
+    assert (a["row_klen"] == b["row_klen"]).all()
+    assert a["cache"]["block_table"] is not None and b["cache"]["block_table"] is None
+    ra = R.dsa_forward_rows(a, range(6))
+    rb = R.dsa_forward_rows(b, range(6))
+    for x, y in zip(ra["scores"], rb["scores"]):
+        np.testing.assert_array_equal(x, y)
+    for x, y in zip(ra["out"], rb["out"]):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_generator_layout_rules():
+    cfg = I.CONFIGS["decode_128k_paged"].replace(ctx_lo=100, ctx_hi=200, n_seqs=4,
+                                                h_idx=2, d_idx=16, n_heads=2, d_c=8, d_r=8)
+    seq, klen = I.row_layout(cfg)
+    ctx = I.context_lengths(cfg)
+    assert list(seq) == [0, 0, 1, 1, 2, 2, 3, 3]
+    assert list(klen) == [int(c) - 1 + j for c in ctx for j in (0, 1)]
+    inp = I.generate(cfg, threads=1)
+    bt = inp["cache"]["block_table"]
+    used = bt[bt >= 0]
+    assert sorted(used) == list(range(inp["cache"]["num_pages"]))   # a permutation
+    # FP8 quantisation: |codes| <= 448 and dequantised keys within one e4m3 step
+    k = R.dequant_keys(inp, np.arange(64))
+    assert np.isfinite(k).all()
+    assert np.abs(R.e4m3_decode(inp["k_idx"])).max() <= 448
+
+
+def test_planted_keys_point_at_their_query():
+    cfg = I.CONFIGS["prefill_8k"].replace(seq_len=256, h_idx=4, plant_frac=0.05)
+    found = 0
+    for blk in range(4):
+        for off, tgt, head in I._plant_targets(cfg, 0, blk):
+            s = blk * 64 + off
+            assert s <= tgt < 256
+            kc, ks, _ = I.key_block(cfg, 0, blk)
+            kv = R.e4m3_decode(kc[off]) * ks[off]
+            qv = I.qidx_rows_f32(cfg, [tgt])[0, head].astype(np.float64)
+            cos = kv @ qv / np.linalg.norm(kv) / np.linalg.norm(qv)
+            assert cos > 0.99 and abs(np.linalg.norm(kv) - 4 * math.sqrt(128)) < 2.0
+            found += 1
+    assert found > 0
