@@ -1,0 +1,212 @@
+/*
+ * dsa.h - C ABI of the B200 DeepSeek Sparse Attention (DSA) forward path.
+ *
+ * The path has three stages, as the DSA description defines them
+ * ("DeepSeek Sparse Attention DSA Architecture Guide"):
+ *
+ *   1. lightning indexer ("Stage 1: The Lightning Indexer", index-score
+ *      equation, generalised to H_I weighted heads):
+ *          I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s]),   s < klen[t]
+ *      with q_I and k_I in FP8 e4m3 and one fp32 scale per query head row and
+ *      per key token ("Native FP8 Precision").
+ *   2. top-k ("Stage 2: Fine-Grained Token Selection and Output Computation",
+ *      selection equation S_t = TopK(I[t,:], k)): the k largest scores, ties
+ *      to the lower position, returned in ascending position order and padded
+ *      with -1 when klen < k (the page's listing clips k to the sequence and
+ *      sorts the positions to keep temporal order).
+ *   3. sparse MLA in absorbed form (same section, output equation; logit of
+ *      "The Classical Multi-Head Latent Attention (MLA) Mechanism"):
+ *          z[i,s] = sm_scale * q[t,i] . (c_s || kR_s),  s in S_t
+ *          out[t,i] = sum_s softmax_s(z[i,:]) * c_s,     lse[t,i] = log sum_s e^z
+ *      The query already carries W_UK; W_UV and the output projection are
+ *      dense GEMMs after this path and are not part of it.
+ *
+ * Conventions (every entry point):
+ *  - All pointers except the dsa_* descriptor structs are DEVICE pointers owned
+ *    by the caller.  The library allocates no device memory: scratch comes from
+ *    the caller's workspace `ws` (size from dsa_workspace_size, 256-byte
+ *    aligned).  Descriptor structs are read on the host during the call only.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  No entry point synchronises, except
+ *    dsa_read_device_status.
+ *  - The return code reports what the host can see: null or misaligned
+ *    pointers, unsupported shapes, a workspace that is too small, CUDA launch
+ *    errors.  Errors found on the device (a block-table entry outside
+ *    [0, num_pages), a bounded wait that ran out) are recorded in a status
+ *    word inside `ws`; read it with dsa_read_device_status.  Nothing traps.
+ *  - Results are deterministic run to run (no floating-point atomics).
+ *  - Row t of a call sees keys s in [0, klen[t]) of sequence row_seq[t].
+ *    Prefill row t of a sequence sees klen = t + 1; decode row j of n_q new
+ *    rows of a sequence with ctx cached tokens sees klen = ctx - (n_q - 1 - j).
+ *  - Top-k indices are logical positions within the sequence.  Only the
+ *    attention stage translates them through the block table.
+ */
+#ifndef DSA_B200_DSA_H_
+#define DSA_B200_DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so callers need no CUDA headers. */
+typedef struct CUstream_st* dsa_stream_t;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, bad layout */
+  DSA_ERR_UNSUPPORTED = 2,   /* shape/dtype combination this build does not run   */
+  DSA_ERR_CUDA = 3,          /* a CUDA call or kernel launch failed               */
+  DSA_ERR_OUT_OF_RANGE = 4,  /* device: block-table entry outside [0, num_pages)   */
+  DSA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out     */
+  DSA_ERR_WORKSPACE = 6      /* ws is NULL, misaligned or smaller than required    */
+} dsa_status;
+
+typedef enum {
+  DSA_F32 = 0,
+  DSA_BF16 = 1,
+  DSA_FP8_E4M3 = 2
+} dsa_dtype;
+
+/* Which kernels to run.  AUTO picks the tensor-core kernels (tcgen05) for the
+ * FP8 indexer with H_I*group <= 256, d_I = 128, and for bf16 MLA with
+ * H = 128, d_c = 512, d_r = 64; everything else runs the SIMT kernels. */
+typedef enum {
+  DSA_ALGO_AUTO = 0,
+  DSA_ALGO_SIMT = 1
+} dsa_algo;
+
+/* Problem dimensions. */
+typedef struct {
+  int32_t n_idx_heads;   /* H_I: indexer heads                          */
+  int32_t d_idx;         /* d_I: indexer head width (bytes per e4m3 key) */
+  int32_t n_heads;       /* H: MLA query heads                          */
+  int32_t d_c;           /* latent width = value width                  */
+  int32_t d_r;           /* decoupled RoPE key width                    */
+  int32_t topk;          /* k, 1 <= k <= 2048                           */
+  dsa_dtype idx_dtype;   /* DSA_FP8_E4M3 (scales required) or DSA_F32   */
+  dsa_dtype mla_dtype;   /* DSA_BF16 or DSA_F32                         */
+  float sm_scale;        /* softmax scale, e.g. 1/sqrt(d_c + d_r)       */
+  dsa_algo algo;
+} dsa_dims;
+
+/* Query rows.  Any mix of sequences. */
+typedef struct {
+  int32_t num_rows;          /* T >= 0                                          */
+  const int32_t* row_seq;    /* [T] device: sequence of row t, in [0, num_seqs)  */
+  const int32_t* row_klen;   /* [T] device: visible keys of row t, in [0, max_klen] */
+  int32_t max_klen;          /* host: upper bound of row_klen (sizes the grid)   */
+  int32_t q_group;           /* 1, 2 or 4: rows [g*q_group, (g+1)*q_group) belong
+                                to one sequence; the indexer scores such a group
+                                against one pass over its keys.  A group that
+                                mixes sequences is reported as
+                                DSA_ERR_INVALID_ARG in the device status word.  */
+} dsa_rows;
+
+/* The two caches of the layer: the latent cache (c || kR per token) and the
+ * indexer key cache (k_I per token + its fp32 scale).  Physical row of logical
+ * key s of sequence b:
+ *   paged (block_table != NULL): block_table[b*max_pages_per_seq + s/page_size]
+ *                                * page_size + s % page_size
+ *   contiguous:                  seq_start[b] + s   (seq_start NULL: s)        */
+typedef struct {
+  const void* latent;         /* [num_tokens, d_c + d_r] bf16 | f32, row-major  */
+  const void* idx_k;          /* [num_tokens, d_idx] e4m3 | f32, row-major      */
+  const float* idx_k_scale;   /* [num_tokens] (required for e4m3, else NULL)     */
+  const int32_t* seq_start;   /* [num_seqs] or NULL (contiguous layout)          */
+  const int32_t* block_table; /* [num_seqs, max_pages_per_seq] or NULL           */
+  int32_t page_size;          /* paged: tokens per page, a multiple of 64        */
+  int32_t max_pages_per_seq;  /* paged: row stride of block_table                */
+  int32_t num_seqs;
+  int64_t num_tokens;         /* rows of latent / idx_k (paged: num_pages*page)  */
+} dsa_cache;
+
+typedef enum {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_MLA = 2,
+  DSA_OP_DECODE_STEP = 3,
+  DSA_OP_FORWARD = 4
+} dsa_op;
+
+/* Human-readable name of a status code (static storage). */
+const char* dsa_status_string(dsa_status s);
+
+/* Text of the last host-side error on the calling thread ("" if none). */
+const char* dsa_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t dsa_version(void);
+
+/* Bytes of workspace `op` needs for these dimensions and rows (host only; no
+ * CUDA call).  Returns 0 for invalid arguments. */
+size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op);
+
+/* Zero the device status word at the head of `ws` (async on stream). */
+dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Synchronise `stream`, copy the device status word of `ws` to *status_out
+ * (one of dsa_status) and clear it.  *detail_out (may be NULL) receives the
+ * row or page that raised it, or -1. */
+dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status_out,
+                                  int32_t* detail_out);
+
+/* Stage 1: indexer scores.
+ *   q_idx   [T, H_I, d_I] e4m3 | f32
+ *   q_scale [T, H_I] fp32 (e4m3 only, else NULL): dequantised q = e4m3 * scale
+ *   w       [T, H_I] fp32 head weights
+ *   scores  [T, ld_scores] fp32 out; entries s >= klen[t] are left unspecified.
+ *           ld_scores >= max_klen and a multiple of 4.
+ * The scale factors are folded exactly: I = k_scale[s] * sum_j (w*q_scale)[t,j]
+ * * ReLU(q8 . k8), since both scales are positive and ReLU is positively
+ * homogeneous. */
+dsa_status dsa_indexer_scores(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                              const void* q_idx, const float* q_scale, const float* w,
+                              float* scores, int64_t ld_scores,
+                              void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Stage 2: top-k selection.
+ *   scores [T, ld_scores] fp32 (only s < klen[t] is read)
+ *   idx    [T, topk] int32 out: ascending logical positions, -1 padded.
+ * Comparison is on the fp32 value (-0.0 == +0.0); equal values go to the
+ * lower position.  NaN scores are unsupported. */
+dsa_status dsa_topk(const dsa_dims* dims, const dsa_rows* rows, const float* scores,
+                    int64_t ld_scores, int32_t* idx, void* ws, size_t ws_bytes,
+                    dsa_stream_t stream);
+
+/* Stage 3: sparse absorbed MLA over the selected rows.
+ *   q   [T, H, d_c + d_r] bf16 | f32
+ *   idx [T, topk] int32 logical positions (entries < 0 are skipped; entries
+ *       >= klen[t] are a caller error and are read as given)
+ *   out [T, H, d_c] bf16 | f32 (same dtype as q)
+ *   lse [T, H] fp32 natural-log sum of exp(z) (may be NULL); -inf and out = 0
+ *       for a row with no selected key. */
+dsa_status dsa_sparse_mla_fwd(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                              const void* q, const int32_t* idx, void* out, float* lse,
+                              void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* The three stages for a batch of decode rows (few rows per sequence), one
+ * enqueue, no host synchronisation.  Scores and indices live in ws unless
+ * dbg_scores [T, round_up(max_klen,128)] / dbg_idx [T, topk] are given, in
+ * which case they are written there. */
+dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                           const void* q_idx, const float* q_scale, const float* w,
+                           const void* q, void* out, float* lse,
+                           float* dbg_scores, int32_t* dbg_idx,
+                           void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* The three stages for any rows (prefill): rows are processed in chunks whose
+ * score buffer fits the workspace; `idx_out` [T, topk] (may be NULL) receives
+ * the selections. */
+dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                       const void* q_idx, const float* q_scale, const float* w,
+                       const void* q, void* out, float* lse, int32_t* idx_out,
+                       void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_DSA_H_ */

@@ -1,0 +1,436 @@
+// api.cu - the C ABI of the DSA forward path: argument checks, workspace
+// planning, kernel selection and launches.  No entry point allocates device
+// memory or synchronises (except dsa_read_device_status).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "dsa_kernels.cuh"
+
+namespace dsa {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kForwardChunkRows = 512;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+int64_t scores_ld(int max_klen) { return ((int64_t)max_klen + 127) / 128 * 128; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#define CHECK_ARG(cond, ...)          \
+  do {                                \
+    if (!(cond)) {                    \
+      set_error(__VA_ARGS__);         \
+      return DSA_ERR_INVALID_ARG;     \
+    }                                 \
+  } while (0)
+
+dsa_status check_dims(const dsa_dims* d) {
+  CHECK_ARG(d != nullptr, "dims is NULL");
+  CHECK_ARG(d->n_idx_heads > 0 && d->d_idx > 0 && d->n_heads > 0 && d->d_c > 0 && d->d_r >= 0,
+            "non-positive dimension");
+  CHECK_ARG(d->topk >= 1 && d->topk <= 2048, "topk %d outside [1, 2048]", d->topk);
+  CHECK_ARG(d->idx_dtype == DSA_FP8_E4M3 || d->idx_dtype == DSA_F32, "idx_dtype must be e4m3 or f32");
+  CHECK_ARG(d->mla_dtype == DSA_BF16 || d->mla_dtype == DSA_F32, "mla_dtype must be bf16 or f32");
+  CHECK_ARG(d->algo == DSA_ALGO_AUTO || d->algo == DSA_ALGO_SIMT, "unknown algo");
+  CHECK_ARG(d->sm_scale > 0.f, "sm_scale must be > 0");
+  if (d->d_idx % 4 != 0 || (d->d_c + d->d_r) % 8 != 0) {
+    set_error("d_idx must be a multiple of 4 and d_c + d_r a multiple of 8");
+    return DSA_ERR_UNSUPPORTED;
+  }
+  return DSA_OK;
+}
+
+dsa_status check_rows(const dsa_rows* r) {
+  CHECK_ARG(r != nullptr, "rows is NULL");
+  CHECK_ARG(r->num_rows >= 0 && r->max_klen >= 0, "negative num_rows or max_klen");
+  CHECK_ARG(r->q_group == 1 || r->q_group == 2 || r->q_group == 4, "q_group must be 1, 2 or 4");
+  if (r->num_rows > 0) {
+    CHECK_ARG(r->row_seq != nullptr && r->row_klen != nullptr, "row_seq / row_klen is NULL");
+  }
+  return DSA_OK;
+}
+
+dsa_status check_cache(const dsa_cache* c, const dsa_dims* d, bool need_idx, bool need_latent) {
+  CHECK_ARG(c != nullptr, "cache is NULL");
+  CHECK_ARG(c->num_seqs > 0 && c->num_tokens >= 0, "cache needs num_seqs > 0");
+  if (need_idx) {
+    CHECK_ARG(c->idx_k != nullptr, "idx_k is NULL");
+    CHECK_ARG(aligned(c->idx_k, 16), "idx_k must be 16-byte aligned");
+    if (d->idx_dtype == DSA_FP8_E4M3) CHECK_ARG(c->idx_k_scale != nullptr, "idx_k_scale is NULL");
+  }
+  if (need_latent) {
+    CHECK_ARG(c->latent != nullptr, "latent is NULL");
+    CHECK_ARG(aligned(c->latent, 16), "latent must be 16-byte aligned");
+  }
+  if (c->block_table) {
+    CHECK_ARG(c->page_size > 0 && c->max_pages_per_seq > 0, "paged cache needs page_size > 0");
+    CHECK_ARG(c->num_tokens % c->page_size == 0, "num_tokens must be num_pages * page_size");
+    CHECK_ARG(c->num_tokens / c->page_size <= INT32_MAX, "too many pages");
+  }
+  return DSA_OK;
+}
+
+CacheMap make_map(const dsa_cache* c) {
+  CacheMap m{};
+  m.seq_start = c->seq_start;
+  m.block_table = c->block_table;
+  m.page_size = c->block_table ? c->page_size : 1;
+  m.page_shift = -1;
+  if (c->block_table && (c->page_size & (c->page_size - 1)) == 0) {
+    int s = 0;
+    while ((1 << s) < c->page_size) ++s;
+    m.page_shift = s;
+  }
+  m.max_pages_per_seq = c->max_pages_per_seq;
+  m.num_pages = c->block_table ? (int32_t)(c->num_tokens / c->page_size) : 0;
+  m.num_tokens = c->num_tokens;
+  return m;
+}
+
+// Workspace layout (offsets from ws, each 256-byte aligned).
+struct WsPlan {
+  size_t status = 0;
+  size_t indexer = 0, indexer_bytes = 0;
+  size_t scores = 0, scores_bytes = 0;
+  size_t idx = 0, idx_bytes = 0;
+  size_t mla = 0, mla_bytes = 0;
+  size_t total = 0;
+  int64_t ld = 0;
+  int chunk_rows = 0;
+  int splits = 1;
+};
+
+WsPlan plan(const dsa_dims* d, const dsa_rows* r, dsa_op op) {
+  WsPlan p;
+  size_t off = kStatusBytes;
+  const int T = r->num_rows;
+  int rows = T;
+  if (op == DSA_OP_FORWARD) rows = T < kForwardChunkRows ? T : kForwardChunkRows;
+  p.chunk_rows = rows;
+  p.ld = scores_ld(r->max_klen);
+  const bool need_idx = op == DSA_OP_INDEXER || op == DSA_OP_DECODE_STEP || op == DSA_OP_FORWARD;
+  const bool need_buf = op == DSA_OP_DECODE_STEP || op == DSA_OP_FORWARD;
+  const bool need_mla = op == DSA_OP_SPARSE_MLA || need_buf;
+  if (need_idx) {
+    p.indexer = off;
+    p.indexer_bytes = align_up(indexer_ws_bytes(rows, r->q_group));
+    off += p.indexer_bytes;
+  }
+  if (need_buf) {
+    p.scores = off;
+    p.scores_bytes = align_up((size_t)rows * (size_t)p.ld * sizeof(float));
+    off += p.scores_bytes;
+    p.idx = off;
+    p.idx_bytes = align_up((size_t)rows * (size_t)d->topk * sizeof(int32_t));
+    off += p.idx_bytes;
+  }
+  if (need_mla) {
+    p.splits = (op == DSA_OP_DECODE_STEP || op == DSA_OP_SPARSE_MLA) ? mla_tc_splits(rows) : 1;
+    p.mla = off;
+    p.mla_bytes = align_up(mla_ws_bytes(rows, d->n_heads, d->d_c, p.splits));
+    off += p.mla_bytes;
+  }
+  p.total = off;
+  return p;
+}
+
+dsa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || !aligned(ws, kAlign)) {
+    set_error("workspace must be non-NULL and 256-byte aligned");
+    return DSA_ERR_WORKSPACE;
+  }
+  if (ws_bytes < need) {
+    set_error("workspace too small: %zu < %zu bytes", ws_bytes, need);
+    return DSA_ERR_WORKSPACE;
+  }
+  return DSA_OK;
+}
+
+uint8_t* at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+IndexerArgs indexer_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c,
+                         const void* q_idx, const float* q_scale, const float* w, float* scores,
+                         int64_t ld, void* ws, const WsPlan& p) {
+  IndexerArgs a{};
+  a.num_rows = r->num_rows;
+  a.max_klen = r->max_klen;
+  a.q_group = r->q_group;
+  a.row_seq = r->row_seq;
+  a.row_klen = r->row_klen;
+  a.n_idx_heads = d->n_idx_heads;
+  a.d_idx = d->d_idx;
+  a.idx_dtype = d->idx_dtype;
+  a.q_idx = q_idx;
+  a.q_scale = q_scale;
+  a.w = w;
+  a.idx_k = c->idx_k;
+  a.idx_k_scale = c->idx_k_scale;
+  a.map = make_map(c);
+  a.scores = scores;
+  a.ld_scores = ld;
+  a.num_seqs = c->num_seqs;
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  a.tile_offsets = reinterpret_cast<int32_t*>(at(ws, p.indexer));
+  return a;
+}
+
+dsa_status run_indexer(const dsa_dims* d, IndexerArgs& a, void* ws, const WsPlan& p,
+                       cudaStream_t s) {
+  if (d->algo == DSA_ALGO_AUTO && indexer_tc_supported(a))
+    return launch_indexer_tc(a, at(ws, p.indexer), p.indexer_bytes, s);
+  return launch_indexer_simt(a, s);
+}
+
+MlaArgs mla_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c, const void* q,
+                 const int32_t* idx, void* out, float* lse, void* ws, const WsPlan& p) {
+  MlaArgs a{};
+  a.num_rows = r->num_rows;
+  a.row_seq = r->row_seq;
+  a.row_klen = r->row_klen;
+  a.n_heads = d->n_heads;
+  a.d_c = d->d_c;
+  a.d_r = d->d_r;
+  a.topk = d->topk;
+  a.mla_dtype = d->mla_dtype;
+  a.sm_scale = d->sm_scale;
+  a.q = q;
+  a.idx = idx;
+  a.latent = c->latent;
+  a.map = make_map(c);
+  a.out = out;
+  a.lse = lse;
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  a.splits = p.splits;
+  a.part_o = reinterpret_cast<float*>(at(ws, p.mla));
+  a.part_ml = a.part_o + (size_t)r->num_rows * p.splits * d->n_heads * d->d_c;
+  return a;
+}
+
+dsa_status run_mla(const dsa_dims* d, MlaArgs& a, cudaStream_t s) {
+  if (d->algo == DSA_ALGO_AUTO && mla_tc_supported(a)) return launch_mla_tc(a, s);
+  return launch_mla_simt(a, s);
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_OUT_OF_RANGE: return "DSA_ERR_OUT_OF_RANGE";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+  }
+  return "DSA_UNKNOWN_STATUS";
+}
+
+const char* dsa_last_error(void) { return g_err; }
+
+int32_t dsa_version(void) { return 100; }
+
+size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op) {
+  if (check_dims(dims) != DSA_OK || check_rows(rows) != DSA_OK) return 0;
+  if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
+  return plan(dims, rows, op).total;
+}
+
+dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  if (check_ws(ws, ws_bytes, kStatusBytes) != DSA_OK) return DSA_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream) != cudaSuccess) {
+    set_error("cudaMemsetAsync failed");
+    return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status_out,
+                                  int32_t* detail_out) {
+  if (status_out == nullptr) {
+    set_error("status_out is NULL");
+    return DSA_ERR_INVALID_ARG;
+  }
+  if (check_ws(ws, kStatusBytes, kStatusBytes) != DSA_OK) return DSA_ERR_WORKSPACE;
+  int32_t h[2] = {0, 0};
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess ||
+      cudaMemsetAsync(ws, 0, kStatusBytes, s) != cudaSuccess) {
+    set_error("reading the device status failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return DSA_ERR_CUDA;
+  }
+  *status_out = h[0];
+  if (detail_out) *detail_out = h[0] ? h[1] : -1;
+  return DSA_OK;
+}
+
+dsa_status dsa_indexer_scores(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                              const void* q_idx, const float* q_scale, const float* w,
+                              float* scores, int64_t ld_scores, void* ws, size_t ws_bytes,
+                              dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows)) ||
+      (st = check_cache(cache, dims, true, false)))
+    return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(q_idx && w && scores, "q_idx / w / scores is NULL");
+    CHECK_ARG(dims->idx_dtype != DSA_FP8_E4M3 || q_scale, "q_scale is NULL for e4m3");
+    CHECK_ARG(aligned(q_idx, 16) && aligned(scores, 16), "q_idx and scores must be 16-byte aligned");
+  }
+  CHECK_ARG(ld_scores >= rows->max_klen && ld_scores % 4 == 0,
+            "ld_scores must be >= max_klen and a multiple of 4");
+  const WsPlan p = plan(dims, rows, DSA_OP_INDEXER);
+  if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  IndexerArgs a = indexer_args(dims, rows, cache, q_idx, q_scale, w, scores, ld_scores, ws, p);
+  return run_indexer(dims, a, ws, p, (cudaStream_t)stream);
+}
+
+dsa_status dsa_topk(const dsa_dims* dims, const dsa_rows* rows, const float* scores,
+                    int64_t ld_scores, int32_t* idx, void* ws, size_t ws_bytes,
+                    dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows))) return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(scores && idx, "scores / idx is NULL");
+    CHECK_ARG(aligned(scores, 16), "scores must be 16-byte aligned");
+  }
+  CHECK_ARG(ld_scores >= rows->max_klen && ld_scores % 4 == 0,
+            "ld_scores must be >= max_klen and a multiple of 4");
+  const WsPlan p = plan(dims, rows, DSA_OP_TOPK);
+  if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  TopkArgs a{};
+  a.num_rows = rows->num_rows;
+  a.row_klen = rows->row_klen;
+  a.scores = scores;
+  a.ld_scores = ld_scores;
+  a.topk = dims->topk;
+  a.idx = idx;
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  return launch_topk(a, rows->max_klen, (cudaStream_t)stream);
+}
+
+dsa_status dsa_sparse_mla_fwd(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                              const void* q, const int32_t* idx, void* out, float* lse, void* ws,
+                              size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows)) ||
+      (st = check_cache(cache, dims, false, true)))
+    return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(q && idx && out, "q / idx / out is NULL");
+    CHECK_ARG(aligned(q, 16) && aligned(out, 16), "q and out must be 16-byte aligned");
+  }
+  const WsPlan p = plan(dims, rows, DSA_OP_SPARSE_MLA);
+  if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  MlaArgs a = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
+  return run_mla(dims, a, (cudaStream_t)stream);
+}
+
+dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                           const void* q_idx, const float* q_scale, const float* w, const void* q,
+                           void* out, float* lse, float* dbg_scores, int32_t* dbg_idx, void* ws,
+                           size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows)) ||
+      (st = check_cache(cache, dims, true, true)))
+    return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(q_idx && w && q && out, "q_idx / w / q / out is NULL");
+    CHECK_ARG(dims->idx_dtype != DSA_FP8_E4M3 || q_scale, "q_scale is NULL for e4m3");
+    CHECK_ARG(aligned(q_idx, 16) && aligned(q, 16) && aligned(out, 16),
+              "q_idx, q and out must be 16-byte aligned");
+    CHECK_ARG(dbg_scores == nullptr || aligned(dbg_scores, 16), "dbg_scores must be 16-byte aligned");
+  }
+  const WsPlan p = plan(dims, rows, DSA_OP_DECODE_STEP);
+  if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  float* scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(at(ws, p.scores));
+  int32_t* idx = dbg_idx ? dbg_idx : reinterpret_cast<int32_t*>(at(ws, p.idx));
+  IndexerArgs ia = indexer_args(dims, rows, cache, q_idx, q_scale, w, scores, p.ld, ws, p);
+  if ((st = run_indexer(dims, ia, ws, p, s))) return st;
+  TopkArgs ta{};
+  ta.num_rows = rows->num_rows;
+  ta.row_klen = rows->row_klen;
+  ta.scores = scores;
+  ta.ld_scores = p.ld;
+  ta.topk = dims->topk;
+  ta.idx = idx;
+  ta.status = reinterpret_cast<DeviceStatus*>(ws);
+  if ((st = launch_topk(ta, rows->max_klen, s))) return st;
+  MlaArgs ma = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
+  return run_mla(dims, ma, s);
+}
+
+dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                       const void* q_idx, const float* q_scale, const float* w, const void* q,
+                       void* out, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes,
+                       dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows)) ||
+      (st = check_cache(cache, dims, true, true)))
+    return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(q_idx && w && q && out, "q_idx / w / q / out is NULL");
+    CHECK_ARG(dims->idx_dtype != DSA_FP8_E4M3 || q_scale, "q_scale is NULL for e4m3");
+    CHECK_ARG(aligned(q_idx, 16) && aligned(q, 16) && aligned(out, 16),
+              "q_idx, q and out must be 16-byte aligned");
+  }
+  const WsPlan p = plan(dims, rows, DSA_OP_FORWARD);
+  if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int T = rows->num_rows;
+  const int H_I = dims->n_idx_heads, D_I = dims->d_idx, H = dims->n_heads;
+  const int DQK = dims->d_c + dims->d_r;
+  const size_t qi_el = dims->idx_dtype == DSA_FP8_E4M3 ? 1 : 4;
+  const size_t mla_el = dims->mla_dtype == DSA_BF16 ? 2 : 4;
+  float* scores = reinterpret_cast<float*>(at(ws, p.scores));
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(at(ws, p.idx));
+  for (int r0 = 0; r0 < T; r0 += p.chunk_rows) {
+    const int n = (T - r0) < p.chunk_rows ? (T - r0) : p.chunk_rows;
+    dsa_rows cr = *rows;
+    cr.num_rows = n;
+    cr.row_seq = rows->row_seq + r0;
+    cr.row_klen = rows->row_klen + r0;
+    const uint8_t* qi = static_cast<const uint8_t*>(q_idx) + (size_t)r0 * H_I * D_I * qi_el;
+    const float* qs = q_scale ? q_scale + (size_t)r0 * H_I : nullptr;
+    const float* wr = w + (size_t)r0 * H_I;
+    const uint8_t* qq = static_cast<const uint8_t*>(q) + (size_t)r0 * H * DQK * mla_el;
+    uint8_t* oo = static_cast<uint8_t*>(out) + (size_t)r0 * H * dims->d_c * mla_el;
+    float* ll = lse ? lse + (size_t)r0 * H : nullptr;
+    int32_t* idx = idx_out ? idx_out + (size_t)r0 * dims->topk : idx_ws;
+    IndexerArgs ia = indexer_args(dims, &cr, cache, qi, qs, wr, scores, p.ld, ws, p);
+    if ((st = run_indexer(dims, ia, ws, p, s))) return st;
+    TopkArgs ta{};
+    ta.num_rows = n;
+    ta.row_klen = cr.row_klen;
+    ta.scores = scores;
+    ta.ld_scores = p.ld;
+    ta.topk = dims->topk;
+    ta.idx = idx;
+    ta.status = reinterpret_cast<DeviceStatus*>(ws);
+    if ((st = launch_topk(ta, rows->max_klen, s))) return st;
+    MlaArgs ma = mla_args(dims, &cr, cache, qq, idx, oo, ll, ws, p);
+    if ((st = run_mla(dims, ma, s))) return st;
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// dsa_kernels.cuh - argument blocks and launchers of the DSA kernels.
+#pragma once
+
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+struct IndexerArgs {
+  int num_rows, max_klen, q_group;
+  const int32_t* row_seq;
+  const int32_t* row_klen;
+  int n_idx_heads, d_idx;
+  dsa_dtype idx_dtype;
+  const void* q_idx;          // [T, H_I, d_I]
+  const float* q_scale;       // [T, H_I] or null
+  const float* w;             // [T, H_I]
+  const void* idx_k;          // [num_tokens, d_I]
+  const float* idx_k_scale;   // [num_tokens] or null
+  CacheMap map;
+  float* scores;
+  int64_t ld_scores;
+  int num_seqs;
+  DeviceStatus* status;
+  int32_t* tile_offsets;      // workspace: [n_groups + 1] exclusive scan of key tiles
+};
+
+struct TopkArgs {
+  int num_rows;
+  const int32_t* row_klen;
+  const float* scores;
+  int64_t ld_scores;
+  int topk;
+  int32_t* idx;               // [T, topk]
+  DeviceStatus* status;
+};
+
+struct MlaArgs {
+  int num_rows;
+  const int32_t* row_seq;
+  const int32_t* row_klen;
+  int n_heads, d_c, d_r, topk;
+  dsa_dtype mla_dtype;
+  float sm_scale;
+  const void* q;              // [T, H, d_c + d_r]
+  const int32_t* idx;         // [T, topk]
+  const void* latent;         // [num_tokens, d_c + d_r]
+  CacheMap map;
+  void* out;                  // [T, H, d_c]
+  float* lse;                 // [T, H] or null
+  DeviceStatus* status;
+  // split-K scratch (tensor-core path)
+  float* part_o;              // [T, splits, H, d_c]
+  float* part_ml;             // [T, splits, H, 2]  (max, sum)
+  int splits;
+};
+
+dsa_status launch_indexer_simt(const IndexerArgs& a, cudaStream_t stream);
+dsa_status launch_indexer_tc(const IndexerArgs& a, void* ws_tail, size_t ws_tail_bytes,
+                             cudaStream_t stream);
+bool indexer_tc_supported(const IndexerArgs& a);
+size_t indexer_ws_bytes(int num_rows, int q_group);
+
+dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream);
+size_t topk_ws_bytes();
+
+dsa_status launch_mla_simt(const MlaArgs& a, cudaStream_t stream);
+dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream);
+bool mla_tc_supported(const MlaArgs& a);
+int mla_tc_splits(int num_rows);
+size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
+
+// Host-side error text of the calling thread.
+void set_error(const char* fmt, ...);
+
+}  // namespace dsa

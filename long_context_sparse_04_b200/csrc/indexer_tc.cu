@@ -1,0 +1,463 @@
+// indexer_tc.cu - FP8 lightning indexer on the 5th-generation tensor cores.
+//
+// Computes, for each query row t and visible key s < klen[t]
+//     I[t,s] = k_scale[s] * sum_j w'[t,j] * ReLU(q8[t,j,:] . k8[s,:]),  w' = w * q_scale
+// which equals sum_j w[t,j] ReLU(q[t,j] . k[s]) on the dequantised operands
+// because both scales are positive and ReLU is positively homogeneous
+// ("DeepSeek Sparse Attention DSA Architecture Guide", section "Stage 1: The
+// Lightning Indexer": index-score equation, FP8 operands).
+//
+// Shape of the contraction: one tile is 128 keys (M) x NQ*64 query-heads (N)
+// x 128 (K = d_I bytes of e4m3).  A query group is NQ consecutive rows of one
+// sequence; all its heads share one pass over the sequence's keys.
+//
+// Roles (persistent CTA, one per SM, 320 threads):
+//   warp 0      TMA producer: 128-key tiles as two 64-row boxes (so a box never
+//               crosses a 64-token page) into a 6-stage ring; the group's
+//               queries (N x 128 B) into a double buffer; w' into smem.
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
+//               into one of two TMEM accumulators (2 x N columns).
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator (lane = key), ReLU,
+//               head-weighted sum with w', times k_scale, coalesced fp32 store.
+// The full L x H_I per-head score tensor lives only in TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "dsa_kernels.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kTileKeys = 128;
+constexpr int kDI = 128;
+constexpr int kHI = 64;
+constexpr int kStages = 6;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kMaxGroups = 2048;
+constexpr int kKeyTileBytes = kTileKeys * kDI;   // 16 KB
+
+template <int NQ>
+struct __align__(1024) IdxSmem {
+  uint8_t keys[kStages][kKeyTileBytes];
+  uint8_t q[2][NQ * kHI * kDI];
+  float wq[2][NQ * kHI];
+  int32_t tile_off[kMaxGroups + 1];
+  int32_t scan_tmp[kThreads / 32];
+  uint64_t full[kStages], empty[kStages];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+};
+
+struct TcArgs {
+  int num_rows, n_groups;
+  const int32_t* row_seq;
+  const int32_t* row_klen;
+  const float* q_scale;
+  const float* w;
+  const float* k_scale;
+  CacheMap map;
+  float* scores;
+  int64_t ld;
+  DeviceStatus* status;
+};
+
+// Walks the flattened (group, key tile) list from a start tile.
+struct TileIter {
+  const int32_t* off;
+  int g, kt, ntiles;
+  __device__ void start(const int32_t* o, int n_groups, int tile) {
+    off = o;
+    int lo = 0, hi = n_groups;            // largest g with off[g] <= tile
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (off[mid] <= tile) lo = mid; else hi = mid;
+    }
+    g = lo;
+    kt = tile - off[g];
+    ntiles = off[g + 1] - off[g];
+  }
+  __device__ void next() {
+    if (++kt >= ntiles) {
+      kt = 0;
+      do { ++g; ntiles = off[g + 1] - off[g]; } while (ntiles == 0);
+    }
+  }
+};
+
+template <int NQ>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                  TcArgs a) {
+  constexpr int N = NQ * kHI;
+  constexpr int kQBytes = N * kDI;
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  IdxSmem<NQ>& S = *reinterpret_cast<IdxSmem<NQ>*>(
+      (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- schedule: exclusive scan of key tiles per group (every CTA, redundantly)
+  {
+    const int chunk = (a.n_groups + kThreads - 1) / kThreads;
+    const int g_lo = min(a.n_groups, (int)threadIdx.x * chunk);
+    const int g_hi = min(a.n_groups, g_lo + chunk);
+    int local = 0;
+    for (int g = g_lo; g < g_hi; ++g) {
+      int mk = 0;
+      const int seq0 = a.row_seq[g * NQ];
+      for (int i = 0; i < NQ; ++i) {
+        const int r = g * NQ + i;
+        if (r < a.num_rows) {
+          mk = max(mk, a.row_klen[r]);
+          if (a.row_seq[r] != seq0) set_status(a.status, DSA_ERR_INVALID_ARG, g);
+        }
+      }
+      const int nt = (mk + kTileKeys - 1) / kTileKeys;
+      S.tile_off[g + 1] = nt;
+      local += nt;
+    }
+    int x = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) S.scan_tmp[warp] = x;
+    __syncthreads();
+    int run = x - local;
+    for (int w2 = 0; w2 < warp; ++w2) run += S.scan_tmp[w2];
+    for (int g = g_lo; g < g_hi; ++g) {
+      run += S.tile_off[g + 1];
+      S.tile_off[g + 1] = run;
+    }
+    if (threadIdx.x == 0) S.tile_off[0] = 0;
+  }
+  if (threadIdx.x == 32) {
+    for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.q_full[i], 1);
+      mbar_init(&S.q_empty[i], 1);
+      mbar_init(&S.acc_full[i], 1);
+      mbar_init(&S.acc_empty[i], kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, 2 * N);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int total = S.tile_off[a.n_groups];
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int t_begin = min(total, (int)blockIdx.x * per);
+  const int t_end = min(total, t_begin + per);
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (lane 0)
+    if (lane == 0 && t_begin < t_end) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_q);
+      TileIter it;
+      it.start(S.tile_off, a.n_groups, t_begin);
+      int qcount = 0, gmax = 0, seq = 0, j = 0;
+      bool alive = true;
+      for (; t_begin + j < t_end; ++j, it.next()) {
+        if (j == 0 || it.kt == 0) {
+          const int qb = qcount & 1;
+          alive = mbar_wait(&S.q_empty[qb], ((qcount >> 1) & 1) ^ 1, a.status, 1);
+          if (!alive) break;
+          const int r0 = it.g * NQ;
+          seq = a.row_seq[r0];
+          gmax = 0;
+          for (int i = 0; i < NQ; ++i)
+            if (r0 + i < a.num_rows) gmax = max(gmax, a.row_klen[r0 + i]);
+          mbar_expect_tx(&S.q_full[qb], kQBytes);
+          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, r0 * kHI);
+          ++qcount;
+        }
+        const int st = j % kStages;
+        alive = mbar_wait(&S.empty[st], ((j / kStages) & 1) ^ 1, a.status, 2);
+        if (!alive) break;
+        int64_t rows[2] = {0, 0};
+        bool load[2];
+        uint32_t bytes = 0;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int s0 = it.kt * kTileKeys + hh * 64;
+          load[hh] = s0 < gmax;
+          if (load[hh]) {
+            bool ok = true;
+            rows[hh] = a.map.row(seq, s0, a.status, &ok);
+            load[hh] = ok;
+          }
+          bytes += load[hh] ? kKeyTileBytes / 2 : 0;
+        }
+        if (bytes == 0) {
+          mbar_arrive(&S.full[st]);
+        } else {
+          mbar_expect_tx(&S.full[st], bytes);
+          for (int hh = 0; hh < 2; ++hh)
+            if (load[hh])
+              tma_load_2d(S.keys[st] + hh * (kKeyTileBytes / 2), &tm_k, &S.full[st], 0,
+                          (int32_t)rows[hh]);
+        }
+      }
+      // tail: wait until the MMAs have released every stage and query buffer in
+      // use, so no commit is still in flight to this CTA's shared memory at exit
+      if (alive) {
+        for (int st = 0; st < kStages && st < j; ++st) {
+          const int last_use = (j - 1 - st) / kStages;
+          if (!mbar_wait(&S.empty[st], last_use & 1, a.status, 7)) break;
+        }
+        for (int qb = 0; qb < 2 && qb < qcount; ++qb) {
+          const int last_use = (qcount - 1 - qb) >> 1;
+          if (!mbar_wait(&S.q_empty[qb], last_use & 1, a.status, 8)) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && t_begin < t_end) {
+      TileIter it;
+      it.start(S.tile_off, a.n_groups, t_begin);
+      constexpr uint32_t idesc = idesc_f8_e4m3(N);
+      int qcount = -1;
+      for (int j = 0; t_begin + j < t_end; ++j) {
+        const bool first = (j == 0 || it.kt == 0);
+        if (first) {
+          ++qcount;
+          if (!mbar_wait(&S.q_full[qcount & 1], (qcount >> 1) & 1, a.status, 3)) break;
+        }
+        const int st = j % kStages, ab = j & 1;
+        if (!mbar_wait(&S.full[st], (j / kStages) & 1, a.status, 4)) break;
+        if (!mbar_wait(&S.acc_empty[ab], ((j >> 1) & 1) ^ 1, a.status, 5)) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(S.keys[st]);
+        const uint32_t qa = smem_u32(S.q[qcount & 1]);
+#pragma unroll
+        for (int k = 0; k < kDI / 32; ++k)
+          mma_f8(tmem + ab * N, sdesc_sw128(ka + 32 * k, 16, 1024), sdesc_sw128(qa + 32 * k, 16, 1024),
+                 idesc, k > 0);
+        mma_commit(&S.empty[st]);
+        mma_commit(&S.acc_full[ab]);
+        const bool last = (it.kt + 1 == it.ntiles) || (t_begin + j + 1 == t_end);
+        if (last) mma_commit(&S.q_empty[qcount & 1]);
+        it.next();
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;               // 0..7
+    const int lq = warp & 3;              // TMEM lane quarter this warp may access
+    const int half = e >> 2;
+    const int row_in_tile = lq * 32 + lane;
+    // queries this warp reduces
+    constexpr int QPW = NQ >= 2 ? NQ / 2 : 1;
+    const bool active = NQ >= 2 || half == 0;
+    TileIter it;
+    if (t_begin < t_end) it.start(S.tile_off, a.n_groups, t_begin);
+    int qcount = -1;
+    int klen[QPW];
+    int seq = 0;
+    for (int j = 0; t_begin + j < t_end; ++j, it.next()) {
+      if (j == 0 || it.kt == 0) {
+        ++qcount;
+        seq = a.row_seq[it.g * NQ];
+        for (int i = 0; i < QPW; ++i) {
+          const int r = it.g * NQ + half * QPW + i;
+          klen[i] = (active && r < a.num_rows) ? a.row_klen[r] : 0;
+        }
+        // w' = w * q_scale of this group into the buffer of this group; the
+        // barrier also guarantees every epilogue thread is done with the group
+        // that used the buffer two groups ago
+        for (int i = threadIdx.x - 64; i < N; i += 32 * kEpiWarps) {
+          const int r = it.g * NQ + i / kHI, h = i % kHI;
+          float v = 0.f;
+          if (r < a.num_rows) v = a.w[(int64_t)r * kHI + h] * a.q_scale[(int64_t)r * kHI + h];
+          S.wq[qcount & 1][i] = v;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory");
+      }
+      const int ab = j & 1;
+      const int qb = qcount & 1;
+      if (!mbar_wait(&S.acc_full[ab], (j >> 1) & 1, a.status, 6)) break;
+      tc_fence_after();
+      const int s = it.kt * kTileKeys + row_in_tile;
+      float res[QPW];
+      if (active) {
+#pragma unroll
+        for (int i = 0; i < QPW; ++i) {
+          const int qi = half * QPW + i;
+          const uint32_t col = tmem + ab * N + qi * kHI + ((uint32_t)(lq * 32) << 16);
+          uint32_t v0[32], v1[32];
+          tmem_ld32(col, v0);
+          tmem_ld32(col + 32, v1);
+          tmem_wait_ld();
+          const float4* wv = reinterpret_cast<const float4*>(&S.wq[qb][qi * kHI]);
+          float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+          for (int h = 0; h < 32; h += 4) {
+            const float4 w0 = wv[h / 4];
+            acc0 = fmaf(fmaxf(__uint_as_float(v0[h + 0]), 0.f), w0.x, acc0);
+            acc1 = fmaf(fmaxf(__uint_as_float(v0[h + 1]), 0.f), w0.y, acc1);
+            acc2 = fmaf(fmaxf(__uint_as_float(v0[h + 2]), 0.f), w0.z, acc2);
+            acc3 = fmaf(fmaxf(__uint_as_float(v0[h + 3]), 0.f), w0.w, acc3);
+            const float4 w1 = wv[8 + h / 4];
+            acc0 = fmaf(fmaxf(__uint_as_float(v1[h + 0]), 0.f), w1.x, acc0);
+            acc1 = fmaf(fmaxf(__uint_as_float(v1[h + 1]), 0.f), w1.y, acc1);
+            acc2 = fmaf(fmaxf(__uint_as_float(v1[h + 2]), 0.f), w1.z, acc2);
+            acc3 = fmaf(fmaxf(__uint_as_float(v1[h + 3]), 0.f), w1.w, acc3);
+          }
+          res[i] = (acc0 + acc1) + (acc2 + acc3);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+      if (active) {
+        int kmax = 0;
+#pragma unroll
+        for (int i = 0; i < QPW; ++i) kmax = max(kmax, klen[i]);
+        if (s < kmax) {
+          bool ok = true;
+          const int64_t pr = a.map.row(seq, s, nullptr, &ok);
+          const float ks = ok ? __ldg(a.k_scale + pr) : 0.f;
+#pragma unroll
+          for (int i = 0; i < QPW; ++i) {
+            const int r = it.g * NQ + half * QPW + i;
+            if (s < klen[i]) a.scores[(int64_t)r * a.ld + s] = res[i] * ks;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * N);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D byte tensor [rows, 128] with 128-byte rows, box 128 x box_rows, 128B swizzle.
+bool make_tmap_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int NQ>
+dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
+  const size_t smem = sizeof(IdxSmem<NQ>) + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(indexer_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess) {
+      set_error("indexer_tc: cannot set %zu bytes of shared memory", smem);
+      return DSA_ERR_CUDA;
+    }
+    attr = true;
+  }
+  CUtensorMap tm_k, tm_q;
+  if (!make_tmap_rows128(&tm_k, a.idx_k, (uint64_t)a.map.num_tokens, 64) ||
+      !make_tmap_rows128(&tm_q, a.q_idx, (uint64_t)a.num_rows * kHI, NQ * kHI)) {
+    set_error("indexer_tc: cuTensorMapEncodeTiled failed");
+    return DSA_ERR_CUDA;
+  }
+  const int n_groups_all = (a.num_rows + NQ - 1) / NQ;
+  for (int g0 = 0; g0 < n_groups_all; g0 += kMaxGroups) {
+    const int ng = min(kMaxGroups, n_groups_all - g0);
+    const int r0 = g0 * NQ;
+    TcArgs t{};
+    t.num_rows = min(a.num_rows - r0, ng * NQ);
+    t.n_groups = ng;
+    t.row_seq = a.row_seq + r0;
+    t.row_klen = a.row_klen + r0;
+    t.q_scale = a.q_scale + (int64_t)r0 * kHI;
+    t.w = a.w + (int64_t)r0 * kHI;
+    t.k_scale = a.idx_k_scale;
+    t.map = a.map;
+    t.scores = a.scores + (int64_t)r0 * a.ld_scores;
+    t.ld = a.ld_scores;
+    t.status = a.status;
+    CUtensorMap tq = tm_q;
+    if (r0 != 0 &&
+        !make_tmap_rows128(&tq, static_cast<const uint8_t*>(a.q_idx) + (int64_t)r0 * kHI * kDI,
+                           (uint64_t)t.num_rows * kHI, NQ * kHI)) {
+      set_error("indexer_tc: cuTensorMapEncodeTiled failed");
+      return DSA_ERR_CUDA;
+    }
+    // upper bound of tiles: groups x ceil(max_klen / 128)
+    const int64_t tiles = (int64_t)ng * ((a.max_klen + kTileKeys - 1) / kTileKeys);
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles));
+    indexer_tc_kernel<NQ><<<grid, kThreads, smem, stream>>>(tm_k, tq, t);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_error("indexer_tc launch: %s", cudaGetErrorString(e));
+      return DSA_ERR_CUDA;
+    }
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+
+bool indexer_tc_supported(const IndexerArgs& a) {
+  if (a.idx_dtype != DSA_FP8_E4M3 || a.d_idx != kDI || a.n_idx_heads != kHI) return false;
+  if (a.q_scale == nullptr || a.idx_k_scale == nullptr) return false;
+  if (a.map.block_table != nullptr && a.map.page_size % 64 != 0) return false;
+  if (a.map.num_tokens >= (int64_t)INT32_MAX) return false;
+  if (encode_fn() == nullptr) return false;
+  return a.q_group == 1 || a.q_group == 2 || a.q_group == 4;
+}
+
+size_t indexer_ws_bytes(int num_rows, int q_group) {
+  return sizeof(int32_t) * (size_t)((num_rows + q_group - 1) / q_group + 1);
+}
+
+dsa_status launch_indexer_tc(const IndexerArgs& a, void*, size_t, cudaStream_t stream) {
+  if (a.num_rows == 0 || a.max_klen == 0) return DSA_OK;
+  switch (a.q_group) {
+    case 1: return launch_nq<1>(a, stream);
+    case 2: return launch_nq<2>(a, stream);
+    default: return launch_nq<4>(a, stream);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,114 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Small workloads with the shapes and distributions of the five configurations
+(several tiles, ragged tails, rows shorter than k), every row checked.
+"""
+import numpy as np
+import pytest
+
+from long_context_sparse_04_b200 import inputs as I
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny_fp32": I.CONFIGS["tiny_fp32"],
+    "decode_small": I.CONFIGS["decode_16k"].replace(ctx_lo=2100, ctx_hi=5000, n_seqs=6),
+    "decode_short_rows": I.CONFIGS["decode_16k"].replace(ctx_lo=1, ctx_hi=2600, n_seqs=8),
+    "prefill_small": I.CONFIGS["prefill_8k"].replace(seq_len=2500),
+    "paged_small": I.CONFIGS["decode_128k_paged"].replace(ctx_lo=2040, ctx_hi=6000, n_seqs=4),
+}
+
+
+@pytest.fixture(scope="module")
+def N():
+    from long_context_sparse_04_b200 import build
+    build.build()
+    from long_context_sparse_04_b200 import _native
+    return _native
+
+
+_cache = {}
+
+
+def _inputs(name):
+    if name not in _cache:
+        _cache[name] = I.generate(SMALL[name])
+    return _cache[name]
+
+
+def _run_stages(N, inp, algo):
+    import torch
+    from long_context_sparse_04_b200.workload import DeviceWorkload
+    wl = DeviceWorkload(inp, algo=algo)
+    scores = wl.indexer()
+    idx = wl.topk_(scores)
+    out, lse = wl.mla(idx)
+    torch.cuda.synchronize()
+    for op in (N.DSA_OP_INDEXER, N.DSA_OP_TOPK, N.DSA_OP_SPARSE_MLA):
+        assert wl.status(op) == (0, -1)
+    return wl, P.to_np(scores), P.to_np(idx), P.to_np(out), P.to_np(lse)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+def test_stagewise_parity(N, name, algo):
+    inp = _inputs(name)
+    a = N.DSA_ALGO_AUTO if algo == "auto" else N.DSA_ALGO_SIMT
+    _, sc, idx, out, lse = _run_stages(N, inp, a)
+    T = inp["row_seq"].shape[0]
+    rows = range(T) if T <= 64 else sorted(set(np.linspace(0, T - 1, 48).astype(int)) | {T - 1})
+    P.check_rows(inp, rows, sc, idx, out, lse)
+
+
+@pytest.mark.parametrize("name", ["decode_small", "paged_small", "tiny_fp32"])
+def test_decode_step_equals_stages(N, name):
+    import torch
+    inp = _inputs(name)
+    wl, sc, idx, out, lse = _run_stages(N, inp, N.DSA_ALGO_AUTO)
+    o2, l2, s2, i2 = wl.decode_step(debug=True)
+    torch.cuda.synchronize()
+    assert wl.status(N.DSA_OP_DECODE_STEP) == (0, -1)
+    klen = inp["row_klen"]
+    s2 = P.to_np(s2)
+    for t in range(len(klen)):
+        assert np.array_equal(s2[t, : klen[t]], sc[t, : klen[t]])
+    assert np.array_equal(P.to_np(i2), idx)
+    np.testing.assert_array_equal(P.to_np(o2), out)
+    np.testing.assert_array_equal(P.to_np(l2), lse)
+
+
+@pytest.mark.parametrize("name", ["prefill_small", "tiny_fp32"])
+def test_forward_equals_stages(N, name):
+    import torch
+    inp = _inputs(name)
+    wl, sc, idx, out, lse = _run_stages(N, inp, N.DSA_ALGO_AUTO)
+    o2, l2, i2 = wl.forward()
+    torch.cuda.synchronize()
+    assert wl.status(N.DSA_OP_FORWARD) == (0, -1)
+    assert np.array_equal(P.to_np(i2), idx)
+    np.testing.assert_array_equal(P.to_np(o2), out)
+
+
+def test_deterministic(N):
+    inp = _inputs("paged_small")
+    a = _run_stages(N, inp, N.DSA_ALGO_AUTO)
+    b = _run_stages(N, inp, N.DSA_ALGO_AUTO)
+    for x, y in zip(a[1:], b[1:]):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_block_table_out_of_range_is_reported(N):
+    import torch
+    from long_context_sparse_04_b200.workload import DeviceWorkload
+    inp = dict(_inputs("paged_small"))
+    cache = dict(inp["cache"])
+    bt = cache["block_table"].copy()
+    bt[1, 3] = cache["num_pages"] + 7          # a page that does not exist
+    cache["block_table"] = bt
+    inp["cache"] = cache
+    wl = DeviceWorkload(inp)
+    wl.indexer()
+    torch.cuda.synchronize()
+    st, det = wl.status(N.DSA_OP_INDEXER)
+    assert st == N.DSA_ERR_OUT_OF_RANGE and det == cache["num_pages"] + 7
