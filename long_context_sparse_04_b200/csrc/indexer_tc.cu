@@ -14,7 +14,7 @@
 // Roles (persistent CTA, one per SM, 320 threads):
 //   warp 0      TMA producer: 128-key tiles as two 64-row boxes (so a box never
 //               crosses a 64-token page) into a 6-stage ring; the group's
-//               queries (N x 128 B) into a double buffer; w' into smem.
+//               queries (N x 128 B) into a double buffer.
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
 //               into one of two TMEM accumulators (2 x N columns).
@@ -42,7 +42,7 @@ template <int NQ>
 struct __align__(1024) IdxSmem {
   uint8_t keys[kStages][kKeyTileBytes];
   uint8_t q[2][NQ * kHI * kDI];
-  float wq[2][NQ * kHI];
+  float wq[kEpiWarps][(NQ >= 2 ? NQ / 2 : 1) * kHI];   // per epilogue warp: w' of its queries
   int32_t tile_off[kMaxGroups + 1];
   int32_t scan_tmp[kThreads / 32];
   uint64_t full[kStages], empty[kStages];
@@ -67,9 +67,10 @@ struct TcArgs {
 // Walks the flattened (group, key tile) list from a start tile.
 struct TileIter {
   const int32_t* off;
-  int g, kt, ntiles;
+  int g, kt, ntiles, ng;
   __device__ void start(const int32_t* o, int n_groups, int tile) {
     off = o;
+    ng = n_groups;
     int lo = 0, hi = n_groups;            // largest g with off[g] <= tile
     while (hi - lo > 1) {
       int mid = (lo + hi) >> 1;
@@ -82,7 +83,10 @@ struct TileIter {
   __device__ void next() {
     if (++kt >= ntiles) {
       kt = 0;
-      do { ++g; ntiles = off[g + 1] - off[g]; } while (ntiles == 0);
+      do {
+        if (++g >= ng) { ntiles = 0; return; }   // past the last tile
+        ntiles = off[g + 1] - off[g];
+      } while (ntiles == 0);
     }
   }
 };
@@ -262,30 +266,28 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const bool active = NQ >= 2 || half == 0;
     TileIter it;
     if (t_begin < t_end) it.start(S.tile_off, a.n_groups, t_begin);
-    int qcount = -1;
     int klen[QPW];
     int seq = 0;
     for (int j = 0; t_begin + j < t_end; ++j, it.next()) {
       if (j == 0 || it.kt == 0) {
-        ++qcount;
         seq = a.row_seq[it.g * NQ];
         for (int i = 0; i < QPW; ++i) {
           const int r = it.g * NQ + half * QPW + i;
           klen[i] = (active && r < a.num_rows) ? a.row_klen[r] : 0;
         }
-        // w' = w * q_scale of this group into the buffer of this group; the
-        // barrier also guarantees every epilogue thread is done with the group
-        // that used the buffer two groups ago
-        for (int i = threadIdx.x - 64; i < N; i += 32 * kEpiWarps) {
-          const int r = it.g * NQ + i / kHI, h = i % kHI;
+        // w' = w * q_scale of this warp's queries into this warp's own slice
+        // (written and read by the same warp: __syncwarp orders it)
+        __syncwarp();
+        for (int i = lane; i < QPW * kHI; i += 32) {
+          const int r = it.g * NQ + half * QPW + i / kHI, h = i % kHI;
           float v = 0.f;
-          if (r < a.num_rows) v = a.w[(int64_t)r * kHI + h] * a.q_scale[(int64_t)r * kHI + h];
-          S.wq[qcount & 1][i] = v;
+          if (active && r < a.num_rows)
+            v = a.w[(int64_t)r * kHI + h] * a.q_scale[(int64_t)r * kHI + h];
+          S.wq[e][i] = v;
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory");
+        __syncwarp();
       }
       const int ab = j & 1;
-      const int qb = qcount & 1;
       if (!mbar_wait(&S.acc_full[ab], (j >> 1) & 1, a.status, 6)) break;
       tc_fence_after();
       const int s = it.kt * kTileKeys + row_in_tile;
@@ -299,7 +301,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           tmem_ld32(col, v0);
           tmem_ld32(col + 32, v1);
           tmem_wait_ld();
-          const float4* wv = reinterpret_cast<const float4*>(&S.wq[qb][qi * kHI]);
+          const float4* wv = reinterpret_cast<const float4*>(&S.wq[e][i * kHI]);
           float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
           for (int h = 0; h < 32; h += 4) {

@@ -17,6 +17,9 @@ SMALL = {
     "decode_short_rows": I.CONFIGS["decode_16k"].replace(ctx_lo=1, ctx_hi=2600, n_seqs=8),
     "prefill_small": I.CONFIGS["prefill_8k"].replace(seq_len=2500),
     "paged_small": I.CONFIGS["decode_128k_paged"].replace(ctx_lo=2040, ctx_hi=6000, n_seqs=4),
+    # rows longer than one CTA's shared-memory segment: top-k runs as a 2-4 CTA cluster
+    "decode_cluster": I.CONFIGS["decode_16k"].replace(ctx_lo=17000, ctx_hi=40000, n_seqs=3),
+    "paged_cluster": I.CONFIGS["decode_128k_paged"].replace(ctx_lo=30000, ctx_hi=70000, n_seqs=2),
 }
 
 
