@@ -1,0 +1,386 @@
+"""Benchmark of the DSA forward hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_128k_paged]
+
+A step is one pass of all three stages (indexer -> top-k -> sparse MLA) over
+one batch of the workload: for the default 128K paged decode workload, 16
+sequences x 2 query rows with contexts drawn from [98304, 131072], one
+dsa_decode_step call.  The metric is query-tokens/s of one DSA layer.
+
+Under torchrun each rank runs its own batch (different seed, same shapes):
+weak scaling, no collective on the data path; the barrier and the max over
+ranks of the device time are the only cross-rank steps.
+
+`--impl reference` times the float64 CPU oracle (the only reference this
+method has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA layer query-tokens/s at 128K decode & 64K prefill; % of roofline"
+UNIT = "query-tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_128k_paged")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=4, help="oracle rows per CPU-baseline sample")
+    ap.add_argument("--n-seqs", type=int, default=None, help="smaller batch (profiling captures)")
+    return ap.parse_args()
+
+
+def dist_info():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def workload_desc(cfg) -> str:
+    if cfg.prefill:
+        head = f"prefill L={cfg.seq_len}"
+    else:
+        head = (f"decode {cfg.n_seqs} seqs x {cfg.rows_per_seq} rows, ctx U[{cfg.ctx_lo},{cfg.ctx_hi}]"
+                + (", 64-token pages, shuffled block table" if cfg.paged else ", contiguous cache"))
+    return (f"{cfg.name}: {head}; indexer H_I={cfg.h_idx} d_I={cfg.d_idx} "
+            f"{'e4m3+per-token fp32 scales' if cfg.fp8 else 'fp32'}; top-k={cfg.topk}; "
+            f"MLA H={cfg.n_heads} d_c={cfg.d_c} d_r={cfg.d_r} {'bf16' if cfg.bf16 else 'fp32'}")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- peaks
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{kernel}@{workload}")
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["sha256"]:
+        return None
+    return d["dram_bytes_per_launch"]
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_rows_per_s(inp, rows, reps=1):
+    from oracle import dsa_ref as R
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        R.dsa_forward_rows(inp, rows)
+    dt = time.perf_counter() - t0
+    return reps * len(rows) / dt, dt
+
+
+def sample_rows(inp, n):
+    import numpy as np
+    T = len(inp["row_seq"])
+    return sorted(set(np.linspace(0, T - 1, n).astype(int).tolist()))
+
+
+def run_reference(args):
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return 0
+    from long_context_sparse_04_b200 import inputs as I
+    cfg = I.CONFIGS[args.workload]
+    inp = I.generate(cfg, with_q=True)
+    rows = sample_rows(inp, 1)
+    cores = len(os.sched_getaffinity(0))
+    for _ in range(args.warmup):
+        oracle_rows_per_s(inp, rows[:1])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_rows_per_s(inp, rows)
+    dt = time.perf_counter() - t0
+    value = args.steps * len(rows) / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_desc(cfg)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{len(rows)} of {len(inp['row_seq'])} query rows per step "
+                                   f"(all three stages, float64 NumPy)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def algorithmic(cfg, inp, stage):
+    """Algorithmic bytes / FLOPs of one launch of a stage on this batch."""
+    import numpy as np
+    klen = inp["row_klen"].astype(np.int64)
+    seqs = inp["row_seq"]
+    T = len(klen)
+    if stage == "indexer":
+        # keys of each sequence read once for all its rows: 128 B e4m3 + 4 B scale per key
+        per_seq = {}
+        for s, k in zip(seqs, klen):
+            per_seq[int(s)] = max(per_seq.get(int(s), 0), int(k))
+        by = sum(per_seq.values()) * (cfg.d_idx + 4)
+        fl = 2 * cfg.h_idx * cfg.d_idx * int(klen.sum())
+        return {"bytes": by, "flops": fl}
+    if stage == "topk":
+        return {"bytes": int(klen.sum()) * 4 + T * cfg.topk * 4, "flops": 0}
+    sel = np.minimum(klen, cfg.topk)
+    by = int(sel.sum()) * cfg.d_qk * 2 + T * cfg.n_heads * (cfg.d_qk + cfg.d_c) * 2
+    fl = int(sel.sum()) * 2 * cfg.n_heads * (cfg.d_qk + cfg.d_c)
+    return {"bytes": by, "flops": fl}
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    rank, world, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from long_context_sparse_04_b200 import build
+    build.build()
+    from long_context_sparse_04_b200 import _native as N
+    from long_context_sparse_04_b200 import inputs as I
+    from long_context_sparse_04_b200.workload import DeviceWorkload
+
+    cfg = I.CONFIGS[args.workload]
+    if args.n_seqs:
+        cfg = cfg.replace(n_seqs=args.n_seqs)
+    cfg_r = cfg.replace(seed=cfg.seed + 1000 * rank)
+    inp = I.generate(cfg_r)
+    wl = DeviceWorkload(inp, device=dev)
+    T = wl.T
+    stream = torch.cuda.current_stream(dev)
+
+    # L2 flush buffer (larger than the 126 MB L2), written before every timed step
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:                 # torch creates the CUDA event on its first record
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    N.dsa_set_stage_events([e.cuda_event for e in ev])
+    out = torch.empty((T, wl.H, wl.d_c), dtype=wl.out_dtype(), device=dev)
+    lse = torch.empty((T, wl.H), dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        wl.decode_step(out=out, lse=lse)
+    torch.cuda.synchronize(dev)
+    st = wl.status(N.DSA_OP_DECODE_STEP)
+    ran = wl.kernels_ran(N.DSA_OP_DECODE_STEP)
+    assert st == (0, -1), f"device status {st}"
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    stage_ms = {"indexer": [], "topk": [], "mla": []}
+    step_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        wl.decode_step(out=out, lse=lse)
+        torch.cuda.synchronize(dev)
+        stage_ms["indexer"].append(ev[0].elapsed_time(ev[1]))
+        stage_ms["topk"].append(ev[1].elapsed_time(ev[2]))
+        stage_ms["mla"].append(ev[2].elapsed_time(ev[3]))
+        step_ms.append(ev[0].elapsed_time(ev[3]))
+    barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    N.dsa_set_stage_events([])
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+    launches_per_step = 3 + (1 if ran & N.DSA_KERNEL_MLA_COMBINE else 0)
+
+    # ---- end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("q_idx", "q_scale", "w", "q", "row_klen")}
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0.record(stream)
+            for k, v in host_in.items():
+                getattr(wl, k).copy_(v, non_blocking=True)
+            wl.decode_step(out=out, lse=lse)
+            host_out.copy_(out, non_blocking=True)
+            host_lse.copy_(lse, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                tot += e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([tot], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            tot = float(t.item())
+        e2e = {"value": world * T * args.steps / (tot / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_kind = measured_peaks()
+    avg = {k: statistics.mean(v) for k, v in stage_ms.items()}
+    dom = max(avg, key=avg.get)
+    alg = algorithmic(cfg_r, inp, dom)
+    mla_tc = bool(ran & N.DSA_KERNEL_MLA_TC)
+    if dom == "mla":
+        bound = "tensor"
+        achieved = alg["flops"] / (avg[dom] / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops")
+        unit = "TFLOP/s"
+    else:
+        bound = "hbm"
+        achieved = alg["bytes"] / (avg[dom] / 1e3) / 1e9
+        peak = peaks.get("hbm_gbs")
+        unit = "GB/s"
+    kname = {"indexer": "indexer_tc_kernel", "topk": "topk_kernel",
+             "mla": "mla_tc_kernel" if mla_tc else "mla_simt_kernel"}[dom]
+    roof = {"kernel": kname, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak if peak else None, "peak_source": peak_kind,
+            "traffic": kernel_traffic(kname, args.workload),
+            "algorithmic_per_launch": alg["bytes"] if bound == "hbm" else alg["flops"]}
+    stages = {}
+    for k in avg:
+        a = algorithmic(cfg_r, inp, k)
+        s = avg[k] / 1e3
+        stages[k] = {"us": 1e3 * avg[k], "hbm_gbs": a["bytes"] / s / 1e9,
+                     "tflops": a["flops"] / s / 1e12}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # bounded sample: about 10-20 s of oracle work on the host cores
+        _, t1 = oracle_rows_per_s(inp, sample_rows(inp, 1))
+        n = int(max(1, min(T, 12.0 / max(t1, 1e-3))))
+        reps = int(max(1, min(8, 12.0 / max(t1 * n, 1e-3))))
+        rows = sample_rows(inp, n)
+        v, dt = oracle_rows_per_s(inp, rows, reps)
+        cpu = {"value": v, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"{len(rows)} of {T} query rows of one batch x {reps}, all three "
+                         f"stages, float64 NumPy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "rows_per_gpu": T,
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "parallelism": f"{world} independent ranks (weak scaling)"},
+            "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

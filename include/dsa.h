@@ -153,6 +153,25 @@ dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream);
 dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status_out,
                                   int32_t* detail_out);
 
+/* Kernel trace: every kernel sets its bit in the workspace's status block when
+ * it runs, so a caller (or a test) can tell which implementation ran. */
+#define DSA_KERNEL_INDEXER_SIMT 0x01u
+#define DSA_KERNEL_INDEXER_TC   0x02u   /* tcgen05 FP8 indexer */
+#define DSA_KERNEL_TOPK         0x04u
+#define DSA_KERNEL_MLA_SIMT     0x08u
+#define DSA_KERNEL_MLA_TC       0x10u   /* tcgen05 bf16 sparse MLA */
+#define DSA_KERNEL_MLA_COMBINE  0x20u   /* split-K combine of the sparse MLA */
+
+/* Synchronise `stream`, return the kernel trace of `ws` in *mask_out and clear it. */
+dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_out);
+
+/* Per-stage timing of dsa_decode_step on the calling thread.  `events` holds
+ * n_events = 4 cudaEvent_t handles created by the caller; each later
+ * dsa_decode_step on this thread records them on its stream before the
+ * indexer, after the indexer, after top-k and after the attention stage.
+ * n_events = 0 turns this off.  The handles are not owned by the library. */
+dsa_status dsa_set_stage_events(void* const* events, int32_t n_events);
+
 /* Stage 1: indexer scores.
  *   q_idx   [T, H_I, d_I] e4m3 | f32
  *   q_scale [T, H_I] fp32 (e4m3 only, else NULL): dequantised q = e4m3 * scale

@@ -15,6 +15,8 @@ DSA_ERR_OUT_OF_RANGE, DSA_ERR_TIMEOUT, DSA_ERR_WORKSPACE = 4, 5, 6
 DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
 DSA_ALGO_AUTO, DSA_ALGO_SIMT = 0, 1
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE_STEP, DSA_OP_FORWARD = range(5)
+DSA_KERNEL_INDEXER_SIMT, DSA_KERNEL_INDEXER_TC, DSA_KERNEL_TOPK = 0x01, 0x02, 0x04
+DSA_KERNEL_MLA_SIMT, DSA_KERNEL_MLA_TC, DSA_KERNEL_MLA_COMBINE = 0x08, 0x10, 0x20
 
 
 class dsa_dims(ctypes.Structure):
@@ -46,6 +48,8 @@ _SIGS = {
     "dsa_workspace_size": (ctypes.c_size_t, [_P, _P, ctypes.c_int]),
     "dsa_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "dsa_read_device_status": (ctypes.c_int, [_P, _P, _P, _P]),
+    "dsa_read_kernel_trace": (ctypes.c_int, [_P, _P, _P]),
+    "dsa_set_stage_events": (ctypes.c_int, [_P, ctypes.c_int32]),
     "dsa_indexer_scores": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
                                           ctypes.c_size_t, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P]),
@@ -101,6 +105,18 @@ def dsa_read_device_status(ws, stream):
     st, det = ctypes.c_int32(0), ctypes.c_int32(0)
     _call("dsa_read_device_status", ws, stream, ctypes.byref(st), ctypes.byref(det))
     return st.value, det.value
+
+
+def dsa_read_kernel_trace(ws, stream) -> int:
+    m = ctypes.c_uint32(0)
+    _call("dsa_read_kernel_trace", ws, stream, ctypes.byref(m))
+    return m.value
+
+
+def dsa_set_stage_events(events):
+    """events: list of 4 raw cudaEvent_t handles (ints), or [] to switch off."""
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e) for e in events]) if events else None
+    return _call("dsa_set_stage_events", arr, len(events))
 
 
 def dsa_indexer_scores(dims, rows, cache, q_idx, q_scale, w, scores, ld_scores, ws, ws_bytes,

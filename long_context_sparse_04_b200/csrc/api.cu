@@ -10,6 +10,12 @@
 namespace dsa {
 
 static thread_local char g_err[512] = "";
+static thread_local cudaEvent_t g_stage_ev[4] = {nullptr, nullptr, nullptr, nullptr};
+static thread_local int g_n_stage_ev = 0;
+
+static void stage_event(int i, cudaStream_t s) {
+  if (g_n_stage_ev == 4 && g_stage_ev[i] != nullptr) cudaEventRecord(g_stage_ev[i], s);
+}
 
 void set_error(const char* fmt, ...) {
   va_list ap;
@@ -273,12 +279,44 @@ dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess ||
-      cudaMemsetAsync(ws, 0, kStatusBytes, s) != cudaSuccess) {
+      cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), s) != cudaSuccess) {
     set_error("reading the device status failed: %s", cudaGetErrorString(cudaGetLastError()));
     return DSA_ERR_CUDA;
   }
   *status_out = h[0];
   if (detail_out) *detail_out = h[0] ? h[1] : -1;
+  return DSA_OK;
+}
+
+dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_out) {
+  if (mask_out == nullptr) {
+    set_error("mask_out is NULL");
+    return DSA_ERR_INVALID_ARG;
+  }
+  if (check_ws(ws, kStatusBytes, kStatusBytes) != DSA_OK) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t* dev = &reinterpret_cast<DeviceStatus*>(ws)->ran;
+  uint32_t h = 0;
+  if (cudaMemcpyAsync(&h, dev, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess || cudaMemsetAsync(dev, 0, sizeof(h), s) != cudaSuccess) {
+    set_error("reading the kernel trace failed");
+    return DSA_ERR_CUDA;
+  }
+  *mask_out = h;
+  return DSA_OK;
+}
+
+dsa_status dsa_set_stage_events(void* const* events, int32_t n_events) {
+  if (n_events == 0) {
+    g_n_stage_ev = 0;
+    return DSA_OK;
+  }
+  if (n_events != 4 || events == nullptr) {
+    set_error("dsa_set_stage_events takes 0 or 4 events");
+    return DSA_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < 4; ++i) g_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);
+  g_n_stage_ev = 4;
   return DSA_OK;
 }
 
@@ -365,7 +403,9 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   float* scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(at(ws, p.scores));
   int32_t* idx = dbg_idx ? dbg_idx : reinterpret_cast<int32_t*>(at(ws, p.idx));
   IndexerArgs ia = indexer_args(dims, rows, cache, q_idx, q_scale, w, scores, p.ld, ws, p);
+  stage_event(0, s);
   if ((st = run_indexer(dims, ia, ws, p, s))) return st;
+  stage_event(1, s);
   TopkArgs ta{};
   ta.num_rows = rows->num_rows;
   ta.row_klen = rows->row_klen;
@@ -375,8 +415,11 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   ta.idx = idx;
   ta.status = reinterpret_cast<DeviceStatus*>(ws);
   if ((st = launch_topk(ta, rows->max_klen, s))) return st;
+  stage_event(2, s);
   MlaArgs ma = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
-  return run_mla(dims, ma, s);
+  st = run_mla(dims, ma, s);
+  stage_event(3, s);
+  return st;
 }
 
 dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,

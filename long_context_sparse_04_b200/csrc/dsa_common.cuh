@@ -18,13 +18,19 @@ namespace dsa {
 struct DeviceStatus {
   int32_t code;     // first error wins (atomicCAS from 0)
   int32_t detail;   // row / page / wait site of that error
-  int32_t pad[62];
+  uint32_t ran;     // DSA_KERNEL_* bits of the kernels that ran
+  int32_t pad[61];
 };
 static constexpr size_t kStatusBytes = 256;
 
 __device__ __forceinline__ void set_status(DeviceStatus* st, int code, int detail) {
   if (st == nullptr) return;
   if (atomicCAS(&st->code, 0, code) == 0) atomicExch(&st->detail, detail);
+}
+
+// Block 0, thread 0 of a kernel marks the kernel as run.
+__device__ __forceinline__ void trace_kernel(DeviceStatus* st, uint32_t bit) {
+  if (st != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(&st->ran, bit);
 }
 
 #ifndef DSA_SPIN_LIMIT
@@ -117,6 +123,16 @@ __device__ __forceinline__ void cp_async_16_zfill(void* smem_dst, const void* gm
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
                "l"(gmem_src), "r"(valid ? 16 : 0) : "memory");
 }
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+// Arrive on `bar` once all cp.async issued so far by this thread have landed
+// (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -147,6 +163,12 @@ __device__ __forceinline__ uint32_t mapa(const void* p, uint32_t rank) {
 __device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ void st_dsmem_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -191,6 +213,15 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem desc], 16-bit operands; A is M lanes x K/2 columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
 // Arrive (once) on `bar` when all tcgen05.mma issued so far by this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -225,6 +256,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15]) : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31]) : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -245,6 +286,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= (uint64_t)1 << 46;     // descriptor version (sm_100)
   d |= (uint64_t)2 << 61;     // SWIZZLE_128B
   return d;
+}
+// K-major, 64-byte swizzle: rows of 64 B, 8-row groups `sbo_bytes` (512) apart.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;     // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;     // SWIZZLE_64B
+  return d;
+}
+// Byte offset of 16-byte chunk `j` (0..3) of row `r` in a 64B-swizzled tile (64-byte
+// rows, base 512-byte aligned).
+__host__ __device__ __forceinline__ uint32_t sw64_off(uint32_t r, uint32_t j) {
+  return r * 64u + ((j ^ ((r >> 1) & 3u)) << 4);
 }
 // Instruction descriptors (dense, fp32 accumulate, M = 128).
 __host__ __device__ constexpr uint32_t idesc_f8_e4m3(int n) {
@@ -285,6 +341,11 @@ struct CacheMap {
     if (block_table != nullptr) {
       int pg = page_shift >= 0 ? (s >> page_shift) : s / page_size;
       int off = s - pg * page_size;
+      if (pg >= max_pages_per_seq) {       // klen beyond the block table's width
+        set_status(st, DSA_ERR_OUT_OF_RANGE, s);
+        *ok = false;
+        return 0;
+      }
       int p = __ldg(block_table + (int64_t)b * max_pages_per_seq + pg);
       if (p < 0 || p >= num_pages) {
         set_status(st, DSA_ERR_OUT_OF_RANGE, p);

@@ -11,16 +11,21 @@
 // x 128 (K = d_I bytes of e4m3).  A query group is NQ consecutive rows of one
 // sequence; all its heads share one pass over the sequence's keys.
 //
-// Roles (persistent CTA, one per SM, 320 threads):
-//   warp 0      TMA producer: 128-key tiles as two 64-row boxes (so a box never
-//               crosses a 64-token page) into a 6-stage ring; the group's
-//               queries (N x 128 B) into a double buffer.
+// Persistent CTAs (one per SM) each own a contiguous range of the flattened
+// (group, key tile) list.  A prologue resolves, through the block table, the
+// physical cache row of both 64-key halves of every tile of the range into
+// shared memory, so the loops below never wait on a dependent global load.
+// Roles (320 threads):
+//   warp 0      producer.  Lane 0: TMA of the two 64-row key boxes (a box never
+//               crosses a 64-token page) into a 6-stage ring, and of the group's
+//               queries (N x 128 B) into a double buffer.  All 32 lanes: cp.async
+//               of the tile's 128 per-key scales into an 8-slot ring.
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
 //               into one of two TMEM accumulators (2 x N columns).
 //   warps 2-9   epilogue: tcgen05.ld of the accumulator (lane = key), ReLU,
 //               head-weighted sum with w', times k_scale, coalesced fp32 store.
-// The full L x H_I per-head score tensor lives only in TMEM.
+// The L x H_I per-head score tensor lives only in TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -33,21 +38,26 @@ constexpr int kTileKeys = 128;
 constexpr int kDI = 128;
 constexpr int kHI = 64;
 constexpr int kStages = 6;
+constexpr int kScaleSlots = 8;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 2048;
+constexpr int kMaxCtaTiles = 512;
 constexpr int kKeyTileBytes = kTileKeys * kDI;   // 16 KB
 
 template <int NQ>
 struct __align__(1024) IdxSmem {
   uint8_t keys[kStages][kKeyTileBytes];
   uint8_t q[2][NQ * kHI * kDI];
+  float scales[kScaleSlots][kTileKeys];
   float wq[kEpiWarps][(NQ >= 2 ? NQ / 2 : 1) * kHI];   // per epilogue warp: w' of its queries
+  int32_t tile_row[kMaxCtaTiles][2];                    // physical row of each 64-key half, -1: none
   int32_t tile_off[kMaxGroups + 1];
   int32_t scan_tmp[kThreads / 32];
   uint64_t full[kStages], empty[kStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
   uint32_t tmem_base;
 };
 
@@ -92,6 +102,17 @@ struct TileIter {
 };
 
 template <int NQ>
+__device__ __forceinline__ int group_max_klen(const TcArgs& a, int g) {
+  int mk = 0;
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) {
+    const int r = g * NQ + i;
+    if (r < a.num_rows) mk = max(mk, a.row_klen[r]);
+  }
+  return mk;
+}
+
+template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   TcArgs a) {
@@ -101,6 +122,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   IdxSmem<NQ>& S = *reinterpret_cast<IdxSmem<NQ>*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  trace_kernel(a.status, DSA_KERNEL_INDEXER_TC);
 
   // ---- schedule: exclusive scan of key tiles per group (every CTA, redundantly)
   {
@@ -109,16 +131,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const int g_hi = min(a.n_groups, g_lo + chunk);
     int local = 0;
     for (int g = g_lo; g < g_hi; ++g) {
-      int mk = 0;
       const int seq0 = a.row_seq[g * NQ];
-      for (int i = 0; i < NQ; ++i) {
+      for (int i = 1; i < NQ; ++i) {
         const int r = g * NQ + i;
-        if (r < a.num_rows) {
-          mk = max(mk, a.row_klen[r]);
-          if (a.row_seq[r] != seq0) set_status(a.status, DSA_ERR_INVALID_ARG, g);
-        }
+        if (r < a.num_rows && a.row_seq[r] != seq0) set_status(a.status, DSA_ERR_INVALID_ARG, g);
       }
-      const int nt = (mk + kTileKeys - 1) / kTileKeys;
+      const int nt = (group_max_klen<NQ>(a, g) + kTileKeys - 1) / kTileKeys;
       S.tile_off[g + 1] = nt;
       local += nt;
     }
@@ -146,6 +164,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       mbar_init(&S.acc_full[i], 1);
       mbar_init(&S.acc_empty[i], kEpiWarps);
     }
+    for (int i = 0; i < kScaleSlots; ++i) {
+      mbar_init(&S.sc_full[i], 32);          // one cp.async arrival per producer lane
+      mbar_init(&S.sc_empty[i], kEpiWarps);
+    }
     fence_mbar_init();
   }
   __syncwarp();
@@ -161,60 +183,77 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const int per = (total + gridDim.x - 1) / gridDim.x;
   const int t_begin = min(total, (int)blockIdx.x * per);
   const int t_end = min(total, t_begin + per);
+  const int ntile = t_end - t_begin;
   const uint32_t tmem = S.tmem_base;
+  if (ntile > kMaxCtaTiles) {           // the host sizes the grid so this cannot happen
+    set_status(a.status, DSA_ERR_INVALID_ARG, -2);
+  } else {
+    // ---- physical rows of both halves of every tile of this CTA's range
+    for (int i = threadIdx.x; i < 2 * ntile; i += kThreads) {
+      TileIter it;
+      it.start(S.tile_off, a.n_groups, t_begin + (i >> 1));
+      const int s0 = it.kt * kTileKeys + (i & 1) * 64;
+      int row = -1;
+      if (s0 < group_max_klen<NQ>(a, it.g)) {
+        bool ok = true;
+        const int64_t r = a.map.row(a.row_seq[it.g * NQ], s0, a.status, &ok);
+        row = ok ? (int32_t)r : -1;
+      }
+      S.tile_row[i >> 1][i & 1] = row;
+    }
+  }
+  __syncthreads();
+  const bool run = ntile > 0 && ntile <= kMaxCtaTiles;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (lane 0)
-    if (lane == 0 && t_begin < t_end) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_q);
+    // ------------------------------------------------------------ producer warp
+    if (run) {
+      if (lane == 0) { prefetch_tmap(&tm_k); prefetch_tmap(&tm_q); }
       TileIter it;
       it.start(S.tile_off, a.n_groups, t_begin);
-      int qcount = 0, gmax = 0, seq = 0, j = 0;
+      int qcount = 0, j = 0;
       bool alive = true;
-      for (; t_begin + j < t_end; ++j, it.next()) {
-        if (j == 0 || it.kt == 0) {
-          const int qb = qcount & 1;
-          alive = mbar_wait(&S.q_empty[qb], ((qcount >> 1) & 1) ^ 1, a.status, 1);
-          if (!alive) break;
-          const int r0 = it.g * NQ;
-          seq = a.row_seq[r0];
-          gmax = 0;
-          for (int i = 0; i < NQ; ++i)
-            if (r0 + i < a.num_rows) gmax = max(gmax, a.row_klen[r0 + i]);
-          mbar_expect_tx(&S.q_full[qb], kQBytes);
-          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, r0 * kHI);
-          ++qcount;
-        }
-        const int st = j % kStages;
-        alive = mbar_wait(&S.empty[st], ((j / kStages) & 1) ^ 1, a.status, 2);
-        if (!alive) break;
-        int64_t rows[2] = {0, 0};
-        bool load[2];
-        uint32_t bytes = 0;
-        for (int hh = 0; hh < 2; ++hh) {
-          const int s0 = it.kt * kTileKeys + hh * 64;
-          load[hh] = s0 < gmax;
-          if (load[hh]) {
-            bool ok = true;
-            rows[hh] = a.map.row(seq, s0, a.status, &ok);
-            load[hh] = ok;
+      for (; j < ntile; ++j, it.next()) {
+        const int st = j % kStages, sl = j % kScaleSlots;
+        if (lane == 0) {
+          if (j == 0 || it.kt == 0) {
+            const int qb = qcount & 1;
+            alive = mbar_wait(&S.q_empty[qb], ((qcount >> 1) & 1) ^ 1, a.status, 1);
+            if (alive) {
+              mbar_expect_tx(&S.q_full[qb], kQBytes);
+              tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, it.g * NQ * kHI);
+            }
           }
-          bytes += load[hh] ? kKeyTileBytes / 2 : 0;
+          alive = alive && mbar_wait(&S.empty[st], ((j / kStages) & 1) ^ 1, a.status, 2);
+          if (alive) {
+            const int r0 = S.tile_row[j][0], r1 = S.tile_row[j][1];
+            const uint32_t bytes = (r0 >= 0 ? kKeyTileBytes / 2 : 0) + (r1 >= 0 ? kKeyTileBytes / 2 : 0);
+            if (bytes == 0) {
+              mbar_arrive(&S.full[st]);
+            } else {
+              mbar_expect_tx(&S.full[st], bytes);
+              if (r0 >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, r0);
+              if (r1 >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, r1);
+            }
+          }
+          alive = alive && mbar_wait(&S.sc_empty[sl], ((j / kScaleSlots) & 1) ^ 1, a.status, 9);
         }
-        if (bytes == 0) {
-          mbar_arrive(&S.full[st]);
-        } else {
-          mbar_expect_tx(&S.full[st], bytes);
-          for (int hh = 0; hh < 2; ++hh)
-            if (load[hh])
-              tma_load_2d(S.keys[st] + hh * (kKeyTileBytes / 2), &tm_k, &S.full[st], 0,
-                          (int32_t)rows[hh]);
+        if (j == 0 || it.kt == 0) ++qcount;
+        alive = __shfl_sync(0xffffffffu, alive, 0);
+        if (!alive) break;
+        // the tile's 128 key scales: 4 per lane, asynchronously
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int k = i * 32 + lane;
+          const int r = S.tile_row[j][k >> 6];
+          if (r >= 0 && (int64_t)r + (k & 63) < a.map.num_tokens)
+            cp_async_4(&S.scales[sl][k], a.k_scale + (int64_t)r + (k & 63));
         }
+        cp_async_mbar_arrive(&S.sc_full[sl]);
       }
       // tail: wait until the MMAs have released every stage and query buffer in
       // use, so no commit is still in flight to this CTA's shared memory at exit
-      if (alive) {
+      if (alive && lane == 0) {
         for (int st = 0; st < kStages && st < j; ++st) {
           const int last_use = (j - 1 - st) / kStages;
           if (!mbar_wait(&S.empty[st], last_use & 1, a.status, 7)) break;
@@ -224,15 +263,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           if (!mbar_wait(&S.q_empty[qb], last_use & 1, a.status, 8)) break;
         }
       }
+      cp_async_wait<0>();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && t_begin < t_end) {
+    if (lane == 0 && run) {
       TileIter it;
       it.start(S.tile_off, a.n_groups, t_begin);
       constexpr uint32_t idesc = idesc_f8_e4m3(N);
       int qcount = -1;
-      for (int j = 0; t_begin + j < t_end; ++j) {
+      for (int j = 0; j < ntile; ++j) {
         const bool first = (j == 0 || it.kt == 0);
         if (first) {
           ++qcount;
@@ -250,27 +290,24 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                  idesc, k > 0);
         mma_commit(&S.empty[st]);
         mma_commit(&S.acc_full[ab]);
-        const bool last = (it.kt + 1 == it.ntiles) || (t_begin + j + 1 == t_end);
+        const bool last = (it.kt + 1 == it.ntiles) || (j + 1 == ntile);
         if (last) mma_commit(&S.q_empty[qcount & 1]);
         it.next();
       }
     }
-  } else {
+  } else if (run) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - 2;               // 0..7
     const int lq = warp & 3;              // TMEM lane quarter this warp may access
     const int half = e >> 2;
     const int row_in_tile = lq * 32 + lane;
-    // queries this warp reduces
-    constexpr int QPW = NQ >= 2 ? NQ / 2 : 1;
+    constexpr int QPW = NQ >= 2 ? NQ / 2 : 1;   // queries this warp reduces
     const bool active = NQ >= 2 || half == 0;
     TileIter it;
-    if (t_begin < t_end) it.start(S.tile_off, a.n_groups, t_begin);
+    it.start(S.tile_off, a.n_groups, t_begin);
     int klen[QPW];
-    int seq = 0;
-    for (int j = 0; t_begin + j < t_end; ++j, it.next()) {
+    for (int j = 0; j < ntile; ++j, it.next()) {
       if (j == 0 || it.kt == 0) {
-        seq = a.row_seq[it.g * NQ];
         for (int i = 0; i < QPW; ++i) {
           const int r = it.g * NQ + half * QPW + i;
           klen[i] = (active && r < a.num_rows) ? a.row_klen[r] : 0;
@@ -287,7 +324,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         __syncwarp();
       }
-      const int ab = j & 1;
+      const int ab = j & 1, sl = j % kScaleSlots;
       if (!mbar_wait(&S.acc_full[ab], (j >> 1) & 1, a.status, 6)) break;
       tc_fence_after();
       const int s = it.kt * kTileKeys + row_in_tile;
@@ -322,19 +359,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
+      if (!mbar_wait(&S.sc_full[sl], (j / kScaleSlots) & 1, a.status, 10)) break;
+      const float ks = S.scales[sl][row_in_tile];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.sc_empty[sl]);
       if (active) {
-        int kmax = 0;
 #pragma unroll
-        for (int i = 0; i < QPW; ++i) kmax = max(kmax, klen[i]);
-        if (s < kmax) {
-          bool ok = true;
-          const int64_t pr = a.map.row(seq, s, nullptr, &ok);
-          const float ks = ok ? __ldg(a.k_scale + pr) : 0.f;
-#pragma unroll
-          for (int i = 0; i < QPW; ++i) {
-            const int r = it.g * NQ + half * QPW + i;
-            if (s < klen[i]) a.scores[(int64_t)r * a.ld + s] = res[i] * ks;
-          }
+        for (int i = 0; i < QPW; ++i) {
+          const int r = it.g * NQ + half * QPW + i;
+          if (s < klen[i]) a.scores[(int64_t)r * a.ld + s] = res[i] * ks;
         }
       }
     }
@@ -396,9 +429,8 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     }
     attr = true;
   }
-  CUtensorMap tm_k, tm_q;
-  if (!make_tmap_rows128(&tm_k, a.idx_k, (uint64_t)a.map.num_tokens, 64) ||
-      !make_tmap_rows128(&tm_q, a.q_idx, (uint64_t)a.num_rows * kHI, NQ * kHI)) {
+  CUtensorMap tm_k;
+  if (!make_tmap_rows128(&tm_k, a.idx_k, (uint64_t)a.map.num_tokens, 64)) {
     set_error("indexer_tc: cuTensorMapEncodeTiled failed");
     return DSA_ERR_CUDA;
   }
@@ -418,16 +450,16 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     t.scores = a.scores + (int64_t)r0 * a.ld_scores;
     t.ld = a.ld_scores;
     t.status = a.status;
-    CUtensorMap tq = tm_q;
-    if (r0 != 0 &&
-        !make_tmap_rows128(&tq, static_cast<const uint8_t*>(a.q_idx) + (int64_t)r0 * kHI * kDI,
+    CUtensorMap tq;
+    if (!make_tmap_rows128(&tq, static_cast<const uint8_t*>(a.q_idx) + (int64_t)r0 * kHI * kDI,
                            (uint64_t)t.num_rows * kHI, NQ * kHI)) {
       set_error("indexer_tc: cuTensorMapEncodeTiled failed");
       return DSA_ERR_CUDA;
     }
-    // upper bound of tiles: groups x ceil(max_klen / 128)
+    // tiles are at most groups x ceil(max_klen / 128); a CTA takes at most kMaxCtaTiles
     const int64_t tiles = (int64_t)ng * ((a.max_klen + kTileKeys - 1) / kTileKeys);
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), tiles));
+    const int64_t need = (tiles + kMaxCtaTiles - 1) / kMaxCtaTiles;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, std::max<int64_t>(num_sms(), need)));
     indexer_tc_kernel<NQ><<<grid, kThreads, smem, stream>>>(tm_k, tq, t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {

@@ -1,9 +1,445 @@
-// mla_tc.cu - tensor-core sparse MLA (placeholder until the tcgen05 kernel lands).
+// mla_tc.cu - sparse absorbed MLA on the 5th-generation tensor cores.
+//
+// For query row t, head i and the selected keys s in S_t ("DeepSeek Sparse
+// Attention DSA Architecture Guide", section "Stage 2: Fine-Grained Token
+// Selection and Output Computation", output equation, in absorbed form):
+//     z[i,s] = sm_scale * q[t,i,:] . (c_s || kR_s)        (576 dims)
+//     out[t,i,:] = sum_s softmax_s(z[i,:]) c_s              (512 dims)
+//
+// Work unit: (row t, key split).  A cluster of two CTAs takes one unit and
+// splits the 576 dims between them: CTA r holds latent dims [256r, 256r+256)
+// and RoPE dims [32r, 32r+32) of Q (128 heads) and of every gathered key.
+//   * S_r = Q_r . KV_r^T (M=128 heads, N=64 keys, K=288) on the tensor cores.
+//   * The two partial logit tiles are exchanged through distributed shared
+//     memory; both CTAs form S = S_0 + S_1 (identical bits) and the same
+//     online softmax, so P is the same in both.
+//   * O_r += P . V_r with V_r = latent dims [256r, 256r+256) of the same
+//     gathered rows (M=128, N=256, K=64), P read from tensor memory.
+// No FLOP is done twice, every gathered byte is read once, and the 128 heads
+// share each gathered row.  The softmax runs in the log2 domain with a lazy
+// rescale: the running max is only moved (and O rescaled) when a block's max
+// exceeds it by more than 8, so P stays <= 256.
+//
+// Roles per CTA (288 threads): warps 0-3 gather (cp.async, 16-byte pieces,
+// swizzled), warps 4-7 softmax / exchange / epilogue (thread = head = TMEM
+// lane), warp 8 TMEM allocation + single-thread MMA issue.
+// TMEM: S double buffer (2 x 64 cols), P double buffer (2 x 32 cols of bf16x2),
+// O (256 cols).
+#include <cuda_bf16.h>
+
 #include "dsa_kernels.cuh"
 
 namespace dsa {
-bool mla_tc_supported(const MlaArgs&) { return false; }
-int mla_tc_splits(int) { return 1; }
-size_t mla_ws_bytes(int, int, int, int) { return 0; }
-dsa_status launch_mla_tc(const MlaArgs&, cudaStream_t) { return DSA_ERR_UNSUPPORTED; }
+namespace {
+
+constexpr int kH = 128, kDC = 512, kDR = 64, kD = kDC + kDR;
+constexpr int kBlk = 64;
+constexpr int kNS = 3;
+constexpr int kMaxKeys = 2048;
+constexpr int kThreads = 32 * 9;
+constexpr int kPieces = 36;                 // 16-byte pieces of one key's 288 dims per CTA
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.0f;
+
+struct __align__(1024) MlaSmem {
+  uint8_t q[4][kH * 128];                   // Q latent dims of this CTA: 4 SW128 chunks of 64 dims
+  uint8_t kv[kNS][4][kBlk * 128];           // gathered latent dims: 4 SW128 chunks x 64 keys
+  uint8_t kv_rope[kNS][kBlk * 64];          // gathered RoPE dims (32), SW64
+  uint8_t q_rope[kH * 64];                  // Q RoPE dims (32), SW64
+  float xbuf[kH * 64];                      // the peer's partial logits, 16-byte pieces swizzled
+  int32_t rows[kMaxKeys];                   // physical cache row per selected key, -1 = none
+  unsigned long long valid[kMaxKeys / kBlk];
+  uint64_t q_full, x_full, x_free;
+  uint64_t kv_full[kNS], kv_empty[kNS];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys_per_split) {
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  MlaSmem& S = *reinterpret_cast<MlaSmem*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const int unit = blockIdx.x >> 1;
+  const int t = unit / a.splits, sp = unit % a.splits;
+  trace_kernel(a.status, DSA_KERNEL_MLA_TC);
+
+  const int klen = a.row_klen[t];
+  const int nsel = min(klen, a.topk);
+  const int k0 = sp * keys_per_split;
+  const int nvalid = max(0, min(nsel - k0, keys_per_split));
+  const int nblk = (nvalid + kBlk - 1) / kBlk;
+  const int seq = a.row_seq[t];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&S.q_full, 128);
+    mbar_init(&S.x_full, 128);
+    mbar_init(&S.x_free, 128);
+    for (int i = 0; i < kNS; ++i) { mbar_init(&S.kv_full[i], 128); mbar_init(&S.kv_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_free[i], 128);
+      mbar_init(&S.p_full[i], 128);
+      mbar_init(&S.pv_done[i], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (warp == 8) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  // physical rows of the selected keys of this split (entries past nvalid are none)
+  const int32_t* idx = a.idx + (int64_t)t * a.topk + k0;
+  for (int i = threadIdx.x; i < nblk * kBlk; i += kThreads) {
+    int row = -1;
+    const int s = i < nvalid ? idx[i] : -1;
+    if (s >= 0 && s < klen) {
+      bool ok = true;
+      const int64_t r = a.map.row(seq, s, a.status, &ok);
+      row = ok ? (int32_t)r : -1;
+    }
+    S.rows[i] = row;
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < nblk; b += kThreads) {
+    unsigned long long m = 0;
+    for (int i = 0; i < kBlk; ++i) m |= (unsigned long long)(S.rows[b * kBlk + i] >= 0) << i;
+    S.valid[b] = m;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync();   // the peer's barriers are initialised before any remote arrive
+  const uint32_t tmem = S.tmem_base;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ gather (128 threads)
+    const int tid = threadIdx.x;
+    if (nblk > 0) {
+      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
+      for (int i = 0; i < kPieces; ++i) {
+        const int qi = i * 128 + tid;
+        const int h = qi / kPieces, c = qi - h * kPieces;
+        if (c < 32) {
+          cp_async_16(S.q[c >> 3] + sw128_off(h, c & 7), qrow + h * kD + 256 * rank + 8 * c);
+        } else {
+          cp_async_16(S.q_rope + sw64_off(h, c - 32), qrow + h * kD + kDC + 32 * rank + 8 * (c - 32));
+        }
+      }
+      cp_async_commit();
+      const __nv_bfloat16* lat = static_cast<const __nv_bfloat16*>(a.latent);
+      bool alive = true;
+      for (int j = 0; j < nblk; ++j) {
+        const int st = j % kNS;
+        if (!mbar_wait(&S.kv_empty[st], ((j / kNS) & 1) ^ 1, a.status, 21)) { alive = false; break; }
+        for (int i = 0; i < (kBlk * kPieces) / 128; ++i) {
+          const int qi = i * 128 + tid;
+          const int key = qi / kPieces, c = qi - key * kPieces;
+          const int row = S.rows[j * kBlk + key];
+          const __nv_bfloat16* src = lat + (int64_t)(row < 0 ? 0 : row) * kD +
+                                     (c < 32 ? 256 * rank + 8 * c : kDC + 32 * rank + 8 * (c - 32));
+          uint8_t* dst = c < 32 ? S.kv[st][c >> 3] + sw128_off(key, c & 7)
+                                : S.kv_rope[st] + sw64_off(key, c - 32);
+          cp_async_16_zfill(dst, src, row >= 0);
+        }
+        cp_async_commit();
+        cp_async_wait<1>();                   // all but the newest group have landed
+        fence_proxy_async_smem();             // make them visible to the tensor cores
+        mbar_arrive(j == 0 ? &S.q_full : &S.kv_full[(j - 1) % kNS]);
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      if (alive) mbar_arrive(&S.kv_full[(nblk - 1) % kNS]);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax / exchange / output
+    const int h = threadIdx.x - 128;                          // head = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c = a.sm_scale * kLog2e;
+    float m_used = -INFINITY, l = 0.f;
+    const uint32_t peer_x = mapa(&S.xbuf[h * 64], peer);
+    bool alive = true;
+    for (int j = 0; j < nblk && alive; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 22)) { alive = false; break; }
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&S.s_free[b]);
+      // exchange partial logits with the peer
+      if (!mbar_wait_cluster(&S.x_free, (j & 1) ^ 1, a.status, 23)) { alive = false; break; }
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4)
+        st_dsmem_v4(peer_x + 16u * (uint32_t)(q4 ^ (h & 15)), v[4 * q4], v[4 * q4 + 1],
+                    v[4 * q4 + 2], v[4 * q4 + 3]);
+      mbar_arrive_cluster(&S.x_full, peer);
+      if (!mbar_wait_cluster(&S.x_full, j & 1, a.status, 24)) { alive = false; break; }
+      float s[64];
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const float4 o = *reinterpret_cast<const float4*>(&S.xbuf[h * 64 + 4 * (q4 ^ (h & 15))]);
+        s[4 * q4 + 0] = __uint_as_float(v[4 * q4 + 0]) + o.x;
+        s[4 * q4 + 1] = __uint_as_float(v[4 * q4 + 1]) + o.y;
+        s[4 * q4 + 2] = __uint_as_float(v[4 * q4 + 2]) + o.z;
+        s[4 * q4 + 3] = __uint_as_float(v[4 * q4 + 3]) + o.w;
+      }
+      mbar_arrive_cluster(&S.x_free, peer);
+      // masked, scaled logits (log2 domain) and the block max
+      const unsigned long long mask = S.valid[j];
+      float mb = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        s[i] = ((mask >> i) & 1ull) ? s[i] * c : -INFINITY;
+        mb = fmaxf(mb, s[i]);
+      }
+      // lazy rescale (warp-uniform because tcgen05.ld/st are warp-collective)
+      const bool need = mb > m_used + kRescale;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? mb : m_used;
+        const float alpha = need ? (m_used == -INFINITY ? 0.f : exp2f(m_used - m_new)) : 1.f;
+        if (j > 0) {
+          if (!mbar_wait(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, 25)) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + kColO + 32 * cc, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem + lane_off + kColO + 32 * cc, o);
+          }
+          tmem_wait_st();
+        }
+        l *= alpha;
+        m_used = m_new;
+      }
+      uint32_t p2[32];
+      float lsum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = (s[2 * i] == -INFINITY) ? 0.f : exp2f(s[2 * i] - m_used);
+        const float p1 = (s[2 * i + 1] == -INFINITY) ? 0.f : exp2f(s[2 * i + 1] - m_used);
+        lsum += p0 + p1;
+        p2[i] = pack_bf16x2(p0, p1);
+      }
+      l += lsum;
+      // P buffer b is free once the PV of block j-2 is done
+      if (!mbar_wait(&S.pv_done[b], ((j >> 1) & 1) ^ 1, a.status, 26)) { alive = false; break; }
+      tc_fence_after();
+      tmem_st32(tmem + lane_off + kColP + b * 32, p2);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&S.p_full[b]);
+    }
+    // ---- output
+    const int64_t ro = ((int64_t)t * kH + h);
+    if (alive && nblk > 0) {
+      alive = mbar_wait(&S.pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, 27);
+      tc_fence_after();
+    }
+    const bool have = alive && nblk > 0;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int cc = 0; cc < 8; ++cc) {
+      uint32_t o[32];
+      if (have) {
+        tmem_ld32(tmem + lane_off + kColO + 32 * cc, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (a.splits > 1) {
+        float4* dst = reinterpret_cast<float4*>(
+            a.part_o + (((int64_t)t * a.splits + sp) * kH + h) * kDC + 256 * rank + 32 * cc);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                               __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ro * kDC +
+                                              256 * rank + 32 * cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float* f = reinterpret_cast<const float*>(&o[8 * i]);
+          dst[i] = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                              pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+        }
+      }
+    }
+    if (rank == 0) {
+      if (a.splits > 1) {
+        reinterpret_cast<float2*>(a.part_ml)[((int64_t)t * a.splits + sp) * kH + h] =
+            make_float2(m_used, l);
+      } else if (a.lse) {
+        a.lse[ro] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nblk > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kBlk, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(256, true);
+      bool ok = mbar_wait(&S.q_full, 0, a.status, 31);
+      const uint32_t qa = smem_u32(S.q[0]), qra = smem_u32(S.q_rope);
+      for (int j = 0; ok && j <= nblk; ++j) {
+        if (j < nblk) {
+          const int st = j % kNS, b = j & 1;
+          if (!(ok = mbar_wait(&S.kv_full[st], (j / kNS) & 1, a.status, 32))) break;
+          if (!(ok = mbar_wait(&S.s_free[b], ((j >> 1) & 1) ^ 1, a.status, 33))) break;
+          tc_fence_after();
+          const uint32_t ka = smem_u32(S.kv[st][0]), kra = smem_u32(S.kv_rope[st]);
+          const uint32_t d = tmem + kColS + b * 64;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(d, sdesc_sw128(qa + ch * kH * 128 + 32 * kk, 16, 1024),
+                       sdesc_sw128(ka + ch * kBlk * 128 + 32 * kk, 16, 1024), idesc_s,
+                       (ch | kk) != 0);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_bf16(d, sdesc_sw64(qra + 32 * kk, 512), sdesc_sw64(kra + 32 * kk, 512), idesc_s, 1);
+          mma_commit(&S.s_full[b]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1, st = jj % kNS, b = jj & 1;
+          if (!(ok = mbar_wait(&S.p_full[b], (jj >> 1) & 1, a.status, 34))) break;
+          tc_fence_after();
+          const uint32_t va = smem_u32(S.kv[st][0]);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem + kColO, tmem + kColP + b * 32 + kk * 8,
+                        sdesc_sw128(va + kk * 16 * 128, kBlk * 128, 1024), idesc_pv,
+                        (jj > 0 || kk > 0));
+          mma_commit(&S.kv_empty[st]);
+          mma_commit(&S.pv_done[b]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // no remote access to this CTA's shared memory is still pending
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// out[t,h,:] = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max_s m_s); fixed split order.
+__global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
+  trace_kernel(a.status, DSA_KERNEL_MLA_COMBINE);
+  const int th = blockIdx.x;
+  const int t = th / kH, h = th % kH;
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
+  float M = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, ml[((int64_t)t * a.splits + s) * kH + h].x);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < a.splits; ++s) {
+    const float2 v = ml[((int64_t)t * a.splits + s) * kH + h];
+    const float w = (v.x == -INFINITY) ? 0.f : exp2f(v.x - M);
+    L += w * v.y;
+    const float4 o = reinterpret_cast<const float4*>(
+        a.part_o + (((int64_t)t * a.splits + s) * kH + h) * kDC)[threadIdx.x];
+    acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + ((int64_t)t * kH + h) * kDC)[threadIdx.x] = pk;
+  if (threadIdx.x == 0 && a.lse) a.lse[(int64_t)t * kH + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+bool mla_tc_supported(const MlaArgs& a) {
+  return a.mla_dtype == DSA_BF16 && a.n_heads == kH && a.d_c == kDC && a.d_r == kDR &&
+         a.topk <= kMaxKeys && a.topk >= 1;
+}
+
+// Key splits of a decode batch: enough (row, split) CTA pairs to cover the SMs once.
+int mla_tc_splits(int num_rows) {
+  if (num_rows <= 0) return 1;
+  const int pairs = sm_count() / 2;
+  int s = 1;
+  while (s < 8 && (int64_t)num_rows * s * 2 <= pairs) s <<= 1;
+  return s;
+}
+
+size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits) {
+  if (splits <= 1) return 0;
+  return (size_t)num_rows * splits * n_heads * (d_c * sizeof(float) + 2 * sizeof(float));
+}
+
+dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
+  if (a.num_rows == 0) return DSA_OK;
+  const size_t smem = sizeof(MlaSmem) + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess) {
+      set_error("mla_tc: cannot set %zu bytes of shared memory", smem);
+      return DSA_ERR_CUDA;
+    }
+    attr = true;
+  }
+  const int keys_per_split = (int)(ceil_div64(ceil_div64(a.topk, a.splits), kBlk) * kBlk);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.num_rows * a.splits * 2));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr2[1];
+  attr2[0].id = cudaLaunchAttributeClusterDimension;
+  attr2[0].val.clusterDim.x = 2;
+  attr2[0].val.clusterDim.y = 1;
+  attr2[0].val.clusterDim.z = 1;
+  cfg.attrs = attr2;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, a, keys_per_split);
+  if (e != cudaSuccess) {
+    set_error("mla_tc launch: %s", cudaGetErrorString(e));
+    return DSA_ERR_CUDA;
+  }
+  if (a.splits > 1) {
+    mla_combine_kernel<<<a.num_rows * kH, 128, 0, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_error("mla_combine launch: %s", cudaGetErrorString(e));
+      return DSA_ERR_CUDA;
+    }
+  }
+  return DSA_OK;
+}
+
 }  // namespace dsa

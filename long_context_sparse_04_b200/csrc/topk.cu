@@ -92,21 +92,37 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t bi
 // Sum the cluster's histograms `which`, then find the bin where the count from
 // the top reaches `need`.  Writes sel_bin / sel_need (need left inside the bin).
 __device__ void select_bin(TopkSmem& S, int which, uint32_t need, uint32_t csize) {
-  constexpr int per = kBins / kThreads;
+  constexpr int per = kBins / kThreads;   // 8 consecutive bins per thread
+  static_assert(per == 8, "two 16-byte loads per CTA");
   uint32_t tot[per];
+  const uint32_t* mine = &S.hist[which][threadIdx.x * per];
+  if (csize == 1) {
+#pragma unroll
+    for (int i = 0; i < per; ++i) tot[i] = mine[i];
+  } else {
+    // issue every remote load first, then add (the loads overlap in flight)
+    uint4 v[8][2];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < (int)csize) {
+        const uint32_t addr = mapa(mine, (uint32_t)r);
+        v[r][0] = ld_dsmem_v4(addr);
+        v[r][1] = ld_dsmem_v4(addr + 16);
+      } else {
+        v[r][0] = v[r][1] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < per; ++i) tot[i] = 0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      tot[0] += v[r][0].x; tot[1] += v[r][0].y; tot[2] += v[r][0].z; tot[3] += v[r][0].w;
+      tot[4] += v[r][1].x; tot[5] += v[r][1].y; tot[6] += v[r][1].z; tot[7] += v[r][1].w;
+    }
+  }
   uint32_t local = 0;
 #pragma unroll
-  for (int i = 0; i < per; ++i) {
-    const int b = threadIdx.x * per + i;
-    uint32_t c = 0;
-    if (csize == 1) {
-      c = S.hist[which][b];
-    } else {
-      for (uint32_t r = 0; r < csize; ++r) c += ld_dsmem_u32(mapa(&S.hist[which][b], r));
-    }
-    tot[i] = c;
-    local += c;
-  }
+  for (int i = 0; i < per; ++i) local += tot[i];
   uint32_t cum = excl_suffix(local, S.scan_tmp[0]);
 #pragma unroll
   for (int i = per - 1; i >= 0; --i) {
@@ -123,6 +139,7 @@ __device__ void select_bin(TopkSmem& S, int which, uint32_t need, uint32_t csize
 __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smraw);
+  trace_kernel(a.status, DSA_KERNEL_TOPK);
   const uint32_t csize = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
   const int t = blockIdx.x / csize;

@@ -6,9 +6,10 @@ indexer, bf16 or fp32 for the MLA side) and lays out the caches (contiguous,
 or 64-token pages under a shuffled block table).  The CUDA path and the CPU
 oracle both receive exactly these bytes.
 
-Every tensor is drawn block by block from
-``numpy.random.Generator(PCG64(SeedSequence([seed, tensor_id, *block])))`` so
-that any query row or any 64-key block can be regenerated alone.
+Every tensor is drawn piece by piece from
+``numpy.random.Generator(PCG64(SeedSequence([seed, tensor_id, *piece])))`` so
+that any query row, or any chunk of 1024 keys (16 pages of 64) of a sequence,
+can be regenerated alone.
 
 The workloads follow the five shapes the pages' DSA description is measured
 at: a tiny fp32 prefill, 8K-16K decode, 8K and 64K causal prefill, and 96K-128K
@@ -28,7 +29,8 @@ import numpy as np
 
 # tensor ids of the seed sequences
 TID_QIDX, TID_W, TID_KIDX, TID_LATENT, TID_Q, TID_PLANT, TID_LEN, TID_TABLE = range(1, 9)
-BLOCK = 64          # key rows per seeded block (also the page size of paged caches)
+BLOCK = 64          # tokens per page of paged caches
+CHUNK = 1024        # keys per seeded chunk of a sequence (a multiple of BLOCK)
 E4M3_MAX = 448.0
 
 
@@ -161,15 +163,15 @@ def q_rows(cfg: DSAConfig, rows) -> np.ndarray:
     return to_bf16_bits(x) if cfg.bf16 else x
 
 
-def _plant_targets(cfg: DSAConfig, seq: int, blk: int):
-    """Planted positions in a 64-key block: list of (offset, target row, target head)."""
+def _plant_targets(cfg: DSAConfig, seq: int, chunk: int):
+    """Planted positions in a 1024-key chunk: list of (offset, target row, target head)."""
     if cfg.plant_frac <= 0:
         return []
-    r = _rng(cfg.seed, TID_PLANT, seq, blk)
-    mask = r.random(BLOCK) < cfg.plant_frac
+    r = _rng(cfg.seed, TID_PLANT, seq, chunk)
+    mask = r.random(CHUNK) < cfg.plant_frac
     out = []
     for off in np.nonzero(mask)[0]:
-        s = blk * BLOCK + int(off)
+        s = chunk * CHUNK + int(off)
         if s >= cfg.seq_len:
             continue
         tgt = int(r.integers(s, cfg.seq_len))
@@ -178,17 +180,17 @@ def _plant_targets(cfg: DSAConfig, seq: int, blk: int):
     return out
 
 
-def key_block(cfg: DSAConfig, seq: int, blk: int):
-    """One 64-key block of both caches for logical keys [64*blk, 64*blk+64).
+def key_chunk(cfg: DSAConfig, seq: int, chunk: int):
+    """Keys [1024*chunk, 1024*chunk + 1024) of sequence `seq`, both caches.
 
-    Returns (k_idx codes or f32 [64, d_I], k_scale [64] or None,
-    latent [64, d_c+d_r] in storage format).
+    Returns (k_idx codes or f32 [1024, d_I], k_scale [1024] or None,
+    latent [1024, d_c+d_r] in storage format).
     """
-    k = _normal(cfg.seed, TID_KIDX, (seq, blk), (BLOCK, cfg.d_idx), cfg.std_kidx)
-    for off, tgt, head in _plant_targets(cfg, seq, blk):
+    k = _normal(cfg.seed, TID_KIDX, (seq, chunk), (CHUNK, cfg.d_idx), cfg.std_kidx)
+    for off, tgt, head in _plant_targets(cfg, seq, chunk):
         qv = qidx_rows_f32(cfg, [tgt])[0, head]
         k[off] = np.float32(4.0 * math.sqrt(cfg.d_idx)) * qv / np.float32(np.linalg.norm(qv))
-    lat = _normal(cfg.seed, TID_LATENT, (seq, blk), (BLOCK, cfg.d_qk), cfg.std_kv)
+    lat = _normal(cfg.seed, TID_LATENT, (seq, chunk), (CHUNK, cfg.d_qk), cfg.std_kv)
     if cfg.fp8:
         kc, ks = to_e4m3_rows(k)
     else:
@@ -263,17 +265,27 @@ def generate(cfg: DSAConfig, with_q: bool = True, threads: int = 8) -> dict:
     k_scale = np.ones(n_tok, dtype=np.float32) if cfg.fp8 else None
     latent = np.zeros((n_tok, cfg.d_qk), dtype=ldt)
 
-    def fill(p):
-        b, lb, phys = p
-        kc, ks, lat = key_block(cfg, b, lb)
-        sl = slice(phys * BLOCK, phys * BLOCK + BLOCK)
-        k_idx[sl] = kc
-        if ks is not None:
-            k_scale[sl] = ks
-        latent[sl] = lat
+    # logical block (seq, lb) -> physical block, then fill chunk by chunk
+    phys_of = {(b, lb): ph for b, lb, ph in placements}
+    per = CHUNK // BLOCK
 
+    def fill(job):
+        b, c = job
+        kc, ks, lat = key_chunk(cfg, b, c)
+        for i in range(per):
+            ph = phys_of.get((b, c * per + i))
+            if ph is None:
+                break
+            src_sl = slice(i * BLOCK, (i + 1) * BLOCK)
+            dst = slice(ph * BLOCK, (ph + 1) * BLOCK)
+            k_idx[dst] = kc[src_sl]
+            if ks is not None:
+                k_scale[dst] = ks[src_sl]
+            latent[dst] = lat[src_sl]
+
+    jobs = [(b, c) for b in range(len(ctx)) for c in range((nblk[b] + per - 1) // per)]
     with ThreadPoolExecutor(max_workers=threads) as ex:
-        list(ex.map(fill, placements))
+        list(ex.map(fill, jobs))
 
     qf = qidx_rows_f32(cfg, range(T))
     if cfg.fp8:

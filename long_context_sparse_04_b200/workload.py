@@ -101,6 +101,10 @@ class DeviceWorkload:
         ws, _ = self.workspace(op)
         return N.dsa_read_device_status(_vp(ws), self.stream)
 
+    def kernels_ran(self, op: int) -> int:
+        ws, _ = self.workspace(op)
+        return N.dsa_read_kernel_trace(_vp(ws), self.stream)
+
     def out_dtype(self):
         return self.torch.bfloat16 if self.mla_bf16 else self.torch.float32
 

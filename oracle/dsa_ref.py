@@ -49,22 +49,29 @@ import numpy as np
 E4M3_EXP_BIAS = 7
 
 
-def e4m3_decode(codes: np.ndarray) -> np.ndarray:
-    """Decode OCP FP8 E4M3 byte codes to float64.
+def _e4m3_value(code: int) -> float:
+    """Value of one OCP FP8 E4M3 code.
 
     Bit layout S EEEE MMM.  Exponent field 0 is subnormal:
     (-1)^S * 2^(1-7) * M/8.  Otherwise (-1)^S * 2^(E-7) * (1 + M/8), except
     E = 15, M = 7, which is NaN (the format has no infinities).
     """
-    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
-    sign = np.where((c >> 7) & 1, -1.0, 1.0)
-    e = (c >> 3) & 0xF
-    m = c & 0x7
-    sub = sign * (2.0 ** (1 - E4M3_EXP_BIAS)) * (m / 8.0)
-    nor = sign * np.ldexp(1.0 + m / 8.0, (e - E4M3_EXP_BIAS).astype(np.int64))
-    out = np.where(e == 0, sub, nor)
-    out = np.where((e == 15) & (m == 7), np.nan, out)
-    return out.astype(np.float64)
+    sign = -1.0 if (code >> 7) & 1 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 15 and m == 7:
+        return float("nan")
+    if e == 0:
+        return sign * 2.0 ** (1 - E4M3_EXP_BIAS) * (m / 8.0)
+    return sign * 2.0 ** (e - E4M3_EXP_BIAS) * (1.0 + m / 8.0)
+
+
+_E4M3_TABLE = np.array([_e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Decode OCP FP8 E4M3 byte codes to float64 (each code through _e4m3_value)."""
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
 
 
 def bf16_decode(bits: np.ndarray) -> np.ndarray:

@@ -20,6 +20,8 @@ SMALL = {
     # rows longer than one CTA's shared-memory segment: top-k runs as a 2-4 CTA cluster
     "decode_cluster": I.CONFIGS["decode_16k"].replace(ctx_lo=17000, ctx_hi=40000, n_seqs=3),
     "paged_cluster": I.CONFIGS["decode_128k_paged"].replace(ctx_lo=30000, ctx_hi=70000, n_seqs=2),
+    # logits with std 8: block maxima move by more than 2^8, so O is rescaled mid-row
+    "decode_sharp": I.CONFIGS["decode_16k"].replace(ctx_lo=2100, ctx_hi=5000, n_seqs=4, std_q=8.0),
 }
 
 
@@ -50,6 +52,17 @@ def _run_stages(N, inp, algo):
     torch.cuda.synchronize()
     for op in (N.DSA_OP_INDEXER, N.DSA_OP_TOPK, N.DSA_OP_SPARSE_MLA):
         assert wl.status(op) == (0, -1)
+    # the intended kernels ran (no silent fallback)
+    ran_idx = wl.kernels_ran(N.DSA_OP_INDEXER)
+    fp8 = inp["idx_dtype"] == "e4m3"
+    want = N.DSA_KERNEL_INDEXER_TC if (fp8 and algo == N.DSA_ALGO_AUTO) else N.DSA_KERNEL_INDEXER_SIMT
+    assert ran_idx == want, hex(ran_idx)
+    assert wl.kernels_ran(N.DSA_OP_TOPK) == N.DSA_KERNEL_TOPK
+    ran_mla = wl.kernels_ran(N.DSA_OP_SPARSE_MLA)
+    if algo == N.DSA_ALGO_SIMT or inp["mla_dtype"] != "bf16":
+        assert ran_mla == N.DSA_KERNEL_MLA_SIMT, hex(ran_mla)
+    else:
+        assert ran_mla & N.DSA_KERNEL_MLA_TC and not ran_mla & N.DSA_KERNEL_MLA_SIMT, hex(ran_mla)
     return wl, P.to_np(scores), P.to_np(idx), P.to_np(out), P.to_np(lse)
 
 
