@@ -172,6 +172,14 @@ dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_o
  * n_events = 0 turns this off.  The handles are not owned by the library. */
 dsa_status dsa_set_stage_events(void* const* events, int32_t n_events);
 
+/* Profiling trace on the calling thread.  When `dev_buf` (device memory,
+ * `bytes` long, zeroed by the caller) is set, the sparse-MLA kernel's first CTA
+ * pair records clock64() stamps of its pipeline events there: int64
+ * [2 CTAs][8 events][32 blocks] (gather issued, gather landed, S issued, PV
+ * issued, logits ready, exchange done, P stored, exchange slot free).
+ * dev_buf = NULL turns it off.  For performance analysis only. */
+dsa_status dsa_set_trace_buffer(void* dev_buf, size_t bytes);
+
 /* Stage 1: indexer scores.
  *   q_idx   [T, H_I, d_I] e4m3 | f32
  *   q_scale [T, H_I] fp32 (e4m3 only, else NULL): dequantised q = e4m3 * scale

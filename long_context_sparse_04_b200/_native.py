@@ -50,6 +50,7 @@ _SIGS = {
     "dsa_read_device_status": (ctypes.c_int, [_P, _P, _P, _P]),
     "dsa_read_kernel_trace": (ctypes.c_int, [_P, _P, _P]),
     "dsa_set_stage_events": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "dsa_set_trace_buffer": (ctypes.c_int, [_P, ctypes.c_size_t]),
     "dsa_indexer_scores": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
                                           ctypes.c_size_t, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P]),
@@ -117,6 +118,10 @@ def dsa_set_stage_events(events):
     """events: list of 4 raw cudaEvent_t handles (ints), or [] to switch off."""
     arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e) for e in events]) if events else None
     return _call("dsa_set_stage_events", arr, len(events))
+
+
+def dsa_set_trace_buffer(buf, nbytes):
+    return _call("dsa_set_trace_buffer", buf, nbytes)
 
 
 def dsa_indexer_scores(dims, rows, cache, q_idx, q_scale, w, scores, ld_scores, ws, ws_bytes,

@@ -13,9 +13,13 @@ static thread_local char g_err[512] = "";
 static thread_local cudaEvent_t g_stage_ev[4] = {nullptr, nullptr, nullptr, nullptr};
 static thread_local int g_n_stage_ev = 0;
 
+static thread_local long long* g_trace = nullptr;
+
 static void stage_event(int i, cudaStream_t s) {
   if (g_n_stage_ev == 4 && g_stage_ev[i] != nullptr) cudaEventRecord(g_stage_ev[i], s);
 }
+
+long long* trace_buffer() { return g_trace; }
 
 void set_error(const char* fmt, ...) {
   va_list ap;
@@ -221,6 +225,7 @@ MlaArgs mla_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c, const
   a.splits = p.splits;
   a.part_o = reinterpret_cast<float*>(at(ws, p.mla));
   a.part_ml = a.part_o + (size_t)r->num_rows * p.splits * d->n_heads * d->d_c;
+  a.trace = trace_buffer();
   return a;
 }
 
@@ -317,6 +322,15 @@ dsa_status dsa_set_stage_events(void* const* events, int32_t n_events) {
   }
   for (int i = 0; i < 4; ++i) g_stage_ev[i] = static_cast<cudaEvent_t>(events[i]);
   g_n_stage_ev = 4;
+  return DSA_OK;
+}
+
+dsa_status dsa_set_trace_buffer(void* dev_buf, size_t bytes) {
+  if (dev_buf != nullptr && bytes < sizeof(long long) * 2 * kTraceEvents * kTraceBlocks) {
+    set_error("trace buffer needs %zu bytes", sizeof(long long) * 2 * kTraceEvents * kTraceBlocks);
+    return DSA_ERR_INVALID_ARG;
+  }
+  g_trace = static_cast<long long*>(dev_buf);
   return DSA_OK;
 }
 

@@ -52,7 +52,12 @@ struct MlaArgs {
   float* part_o;              // [T, splits, H, d_c]
   float* part_ml;             // [T, splits, H, 2]  (max, sum)
   int splits;
+  long long* trace;           // profiling stamps or null
 };
+
+// Profiling trace buffer registered on the calling host thread (or null).
+long long* trace_buffer();
+static constexpr int kTraceEvents = 8, kTraceBlocks = 32;
 
 dsa_status launch_indexer_simt(const IndexerArgs& a, cudaStream_t stream);
 dsa_status launch_indexer_tc(const IndexerArgs& a, void* ws_tail, size_t ws_tail_bytes,

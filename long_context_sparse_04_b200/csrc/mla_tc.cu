@@ -20,9 +20,10 @@
 // rescale: the running max is only moved (and O rescaled) when a block's max
 // exceeds it by more than 8, so P stays <= 256.
 //
-// Roles per CTA (288 threads): warps 0-3 gather (cp.async, 16-byte pieces,
-// swizzled), warps 4-7 softmax / exchange / epilogue (thread = head = TMEM
-// lane), warp 8 TMEM allocation + single-thread MMA issue.
+// Roles per CTA (416 threads): warps 0-3 gather (cp.async, 16-byte pieces,
+// swizzled), warps 4-7 push the partial logits to the peer, warps 8-11 softmax
+// and epilogue (thread = head = TMEM lane), warp 12 TMEM allocation and
+// single-thread MMA issue.
 // TMEM: S double buffer (2 x 64 cols), P double buffer (2 x 32 cols of bf16x2),
 // O (256 cols).
 #include <cuda_bf16.h>
@@ -34,14 +35,15 @@ namespace {
 
 constexpr int kH = 128, kDC = 512, kDR = 64, kD = kDC + kDR;
 constexpr int kBlk = 64;
-constexpr int kNS = 3;
+constexpr int kNS = 2;
 constexpr int kMaxKeys = 2048;
-constexpr int kThreads = 32 * 9;
+constexpr int kThreads = 32 * 13;
 constexpr int kPieces = 36;                 // 16-byte pieces of one key's 288 dims per CTA
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;
+constexpr uint32_t kXBytes = kH * 64 * sizeof(float);   // one exchanged logit tile
 
 struct __align__(1024) MlaSmem {
   uint8_t q[4][kH * 128];                   // Q latent dims of this CTA: 4 SW128 chunks of 64 dims
@@ -49,6 +51,7 @@ struct __align__(1024) MlaSmem {
   uint8_t kv_rope[kNS][kBlk * 64];          // gathered RoPE dims (32), SW64
   uint8_t q_rope[kH * 64];                  // Q RoPE dims (32), SW64
   float xbuf[kH * 64];                      // the peer's partial logits, 16-byte pieces swizzled
+  float sbuf[kH * 64];                      // this CTA's partial logits, bulk-copied to the peer
   int32_t rows[kMaxKeys];                   // physical cache row per selected key, -1 = none
   unsigned long long valid[kMaxKeys / kBlk];
   uint64_t q_full, x_full, x_free;
@@ -60,6 +63,18 @@ struct __align__(1024) MlaSmem {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 2^x with the hardware approximation (ex2.approx.ftz.f32; 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void tstamp(long long* tr, uint32_t rank, int ev, int j) {
+  if (tr != nullptr && blockIdx.x < 2 && j < kTraceBlocks)
+    tr[((int)rank * kTraceEvents + ev) * kTraceBlocks + j] = clock64();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys_per_split) {
@@ -81,19 +96,20 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
 
   if (threadIdx.x == 0) {
     mbar_init(&S.q_full, 128);
-    mbar_init(&S.x_full, 128);
-    mbar_init(&S.x_free, 128);
+    mbar_init(&S.x_full, 1);                 // armed by this CTA, completed by the peer's copy
+    mbar_init(&S.x_free, 1);                 // the peer's receive buffer is free
     for (int i = 0; i < kNS; ++i) { mbar_init(&S.kv_full[i], 128); mbar_init(&S.kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_free[i], 128);
+      mbar_init(&S.s_free[i], 256);         // exchange + softmax warpgroups
       mbar_init(&S.p_full[i], 128);
       mbar_init(&S.pv_done[i], 1);
     }
     fence_mbar_init();
+    if (nblk > 0) mbar_expect_tx(&S.x_full, kXBytes);   // arm the first transfer
   }
   __syncwarp();
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -135,12 +151,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
           cp_async_16(S.q_rope + sw64_off(h, c - 32), qrow + h * kD + kDC + 32 * rank + 8 * (c - 32));
         }
       }
-      cp_async_commit();
+      cp_async_mbar_arrive(&S.q_full);        // arrives when this thread's Q pieces land
       const __nv_bfloat16* lat = static_cast<const __nv_bfloat16*>(a.latent);
       bool alive = true;
       for (int j = 0; j < nblk; ++j) {
         const int st = j % kNS;
         if (!mbar_wait(&S.kv_empty[st], ((j / kNS) & 1) ^ 1, a.status, 21)) { alive = false; break; }
+        if (tid == 0) tstamp(a.trace, rank, 0, j);
         for (int i = 0; i < (kBlk * kPieces) / 128; ++i) {
           const int qi = i * 128 + tid;
           const int key = qi / kPieces, c = qi - key * kPieces;
@@ -151,69 +168,112 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
                                 : S.kv_rope[st] + sw64_off(key, c - 32);
           cp_async_16_zfill(dst, src, row >= 0);
         }
-        cp_async_commit();
-        cp_async_wait<1>();                   // all but the newest group have landed
-        fence_proxy_async_smem();             // make them visible to the tensor cores
-        mbar_arrive(j == 0 ? &S.q_full : &S.kv_full[(j - 1) % kNS]);
+        // arrives when this thread's pieces of block j land; the MMA thread makes
+        // them visible to the tensor cores (proxy fence) after its wait
+        cp_async_mbar_arrive(&S.kv_full[st]);
       }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      if (alive) mbar_arrive(&S.kv_full[(nblk - 1) % kNS]);
+      cp_async_wait_all();
+      (void)alive;
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax / exchange / output
+    // ------------------------------------------------------------ exchange (128 threads)
+    // Copies this CTA's partial logits of block j to the peer with one bulk copy
+    // while the softmax warpgroup is still working on block j-1.  A wait that
+    // times out only marks the warpgroup dead: the named barriers stay uniform.
     const int h = threadIdx.x - 128;                          // head = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    bool dead = false;
+    for (int j = 0; j < nblk; ++j) {
+      const int b = j & 1;
+      uint32_t v[64];
+      dead = dead || !mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 22);
+      if (!dead) {
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&S.s_free[b]);
+      }
+      if (h == 0 && j > 0) bulk_wait_read0();               // the previous copy has left sbuf
+      named_bar_sync(2, 128);
+      if (!dead) {
+#pragma unroll
+        for (int q4 = 0; q4 < 16; ++q4)
+          *reinterpret_cast<uint4*>(&S.sbuf[h * 64 + 4 * (q4 ^ (h & 15))]) =
+              make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+      }
+      fence_proxy_async_smem();                              // sbuf writes -> async copy engine
+      named_bar_sync(2, 128);
+      if (h == 0 && !dead) {
+        if (mbar_wait_cluster(&S.x_free, (j & 1) ^ 1, a.status, 23)) {
+          tstamp(a.trace, rank, 7, j);
+          bulk_copy_to_peer(S.xbuf, S.sbuf, kXBytes, &S.x_full, peer);
+          bulk_commit();
+        }
+      }
+    }
+    if (h == 0) bulk_wait_read0();
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ softmax / output (128 threads)
+    const int h = threadIdx.x - 256;                          // head = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const float c = a.sm_scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
-    const uint32_t peer_x = mapa(&S.xbuf[h * 64], peer);
-    bool alive = true;
-    for (int j = 0; j < nblk && alive; ++j) {
+    // A wait that times out marks the thread dead; the loop is left together
+    // at the named barrier, and warp-collective tcgen05 ops stay uniform.
+    bool dead = false;
+    for (int j = 0; j < nblk; ++j) {
       const int b = j & 1;
-      if (!mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 22)) { alive = false; break; }
+      dead = dead || !mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 28);
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      if (h == 0) tstamp(a.trace, rank, 4, j);
+      float s[64];
+      tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&S.s_free[b]);
-      // exchange partial logits with the peer
-      if (!mbar_wait_cluster(&S.x_free, (j & 1) ^ 1, a.status, 23)) { alive = false; break; }
-#pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4)
-        st_dsmem_v4(peer_x + 16u * (uint32_t)(q4 ^ (h & 15)), v[4 * q4], v[4 * q4 + 1],
-                    v[4 * q4 + 2], v[4 * q4 + 3]);
-      mbar_arrive_cluster(&S.x_full, peer);
-      if (!mbar_wait_cluster(&S.x_full, j & 1, a.status, 24)) { alive = false; break; }
-      float s[64];
+      // the peer's partial logits of this block, then S = own + peer (same bits in both CTAs)
+      dead = dead || !mbar_wait_cluster(&S.x_full, j & 1, a.status, 24);
+      if (h == 0) tstamp(a.trace, rank, 5, j);
 #pragma unroll
       for (int q4 = 0; q4 < 16; ++q4) {
         const float4 o = *reinterpret_cast<const float4*>(&S.xbuf[h * 64 + 4 * (q4 ^ (h & 15))]);
-        s[4 * q4 + 0] = __uint_as_float(v[4 * q4 + 0]) + o.x;
-        s[4 * q4 + 1] = __uint_as_float(v[4 * q4 + 1]) + o.y;
-        s[4 * q4 + 2] = __uint_as_float(v[4 * q4 + 2]) + o.z;
-        s[4 * q4 + 3] = __uint_as_float(v[4 * q4 + 3]) + o.w;
+        s[4 * q4 + 0] += o.x;
+        s[4 * q4 + 1] += o.y;
+        s[4 * q4 + 2] += o.z;
+        s[4 * q4 + 3] += o.w;
       }
-      mbar_arrive_cluster(&S.x_free, peer);
-      // masked, scaled logits (log2 domain) and the block max
+      if (named_bar_or(3, 128, dead)) { dead = true; break; }   // whole tile read, all alive
+      if (h == 0) {
+        if (j + 1 < nblk) mbar_expect_tx(&S.x_full, kXBytes);   // arm the next transfer first
+        mbar_arrive_cluster(&S.x_free, peer);                    // then free the buffer
+      }
+      // masked (only partial blocks), scaled logits in the log2 domain; block max
       const unsigned long long mask = S.valid[j];
-      float mb = -INFINITY;
+      if (mask != ~0ull) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (!((mask >> i) & 1ull)) s[i] = -INFINITY;
+      }
+      float pm[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pm[i] = s[i] * c;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        s[i] = ((mask >> i) & 1ull) ? s[i] * c : -INFINITY;
-        mb = fmaxf(mb, s[i]);
+        s[i] *= c;
+        if (i >= 8) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
       }
+      const float mb = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       // lazy rescale (warp-uniform because tcgen05.ld/st are warp-collective)
       const bool need = mb > m_used + kRescale;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? mb : m_used;
         const float alpha = need ? (m_used == -INFINITY ? 0.f : exp2f(m_used - m_new)) : 1.f;
         if (j > 0) {
-          if (!mbar_wait(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, 25)) {
-            alive = false;
-            break;
-          }
+          dead = dead || !mbar_wait(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, 25);
           tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < 8; ++cc) {
@@ -229,31 +289,35 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         l *= alpha;
         m_used = m_new;
       }
+      // p = 2^(s - m); a masked key (s = -inf) gives 0.  While no key of the row
+      // has been visible, every s is -inf and m is taken as 0.
+      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t p2[32];
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = (s[2 * i] == -INFINITY) ? 0.f : exp2f(s[2 * i] - m_used);
-        const float p1 = (s[2 * i + 1] == -INFINITY) ? 0.f : exp2f(s[2 * i + 1] - m_used);
-        lsum += p0 + p1;
+        const float p0 = ex2_approx(s[2 * i] - mu);
+        const float p1 = ex2_approx(s[2 * i + 1] - mu);
+        ls[i & 3] += p0 + p1;
         p2[i] = pack_bf16x2(p0, p1);
       }
-      l += lsum;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       // P buffer b is free once the PV of block j-2 is done
-      if (!mbar_wait(&S.pv_done[b], ((j >> 1) & 1) ^ 1, a.status, 26)) { alive = false; break; }
+      dead = dead || !mbar_wait(&S.pv_done[b], ((j >> 1) & 1) ^ 1, a.status, 26);
       tc_fence_after();
       tmem_st32(tmem + lane_off + kColP + b * 32, p2);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&S.p_full[b]);
+      if (h == 0) tstamp(a.trace, rank, 6, j);
     }
     // ---- output
     const int64_t ro = ((int64_t)t * kH + h);
-    if (alive && nblk > 0) {
-      alive = mbar_wait(&S.pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, 27);
+    if (!dead && nblk > 0) {
+      dead = !mbar_wait(&S.pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, 27);
       tc_fence_after();
     }
-    const bool have = alive && nblk > 0;
+    const bool have = __all_sync(0xffffffffu, !dead) && nblk > 0;
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
     for (int cc = 0; cc < 8; ++cc) {
@@ -297,11 +361,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       constexpr uint32_t idesc_s = idesc_bf16(kBlk, false);
       constexpr uint32_t idesc_pv = idesc_bf16(256, true);
       bool ok = mbar_wait(&S.q_full, 0, a.status, 31);
+      fence_proxy_async_smem();
       const uint32_t qa = smem_u32(S.q[0]), qra = smem_u32(S.q_rope);
       for (int j = 0; ok && j <= nblk; ++j) {
         if (j < nblk) {
           const int st = j % kNS, b = j & 1;
           if (!(ok = mbar_wait(&S.kv_full[st], (j / kNS) & 1, a.status, 32))) break;
+          fence_proxy_async_smem();           // gathered (generic-proxy) writes -> tensor cores
+          tstamp(a.trace, rank, 1, j);
           if (!(ok = mbar_wait(&S.s_free[b], ((j >> 1) & 1) ^ 1, a.status, 33))) break;
           tc_fence_after();
           const uint32_t ka = smem_u32(S.kv[st][0]), kra = smem_u32(S.kv_rope[st]);
@@ -317,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
           for (int kk = 0; kk < 2; ++kk)
             mma_bf16(d, sdesc_sw64(qra + 32 * kk, 512), sdesc_sw64(kra + 32 * kk, 512), idesc_s, 1);
           mma_commit(&S.s_full[b]);
+          tstamp(a.trace, rank, 2, j);
         }
         if (j >= 1) {
           const int jj = j - 1, st = jj % kNS, b = jj & 1;
@@ -330,6 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
                         (jj > 0 || kk > 0));
           mma_commit(&S.kv_empty[st]);
           mma_commit(&S.pv_done[b]);
+          tstamp(a.trace, rank, 3, jj);
         }
       }
     }
@@ -337,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   tc_fence_before();
   __syncthreads();
   cluster_sync();   // no remote access to this CTA's shared memory is still pending
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
