@@ -15,16 +15,17 @@
 // (group, key tile) list.  A prologue resolves, through the block table, the
 // physical cache row of both 64-key halves of every tile of the range into
 // shared memory, so the loops below never wait on a dependent global load.
-// Roles (320 threads):
-//   warp 0      producer.  Lane 0: TMA of the two 64-row key boxes (a box never
-//               crosses a 64-token page) into a 6-stage ring, and of the group's
-//               queries (N x 128 B) into a double buffer.  All 32 lanes: cp.async
-//               of the tile's 128 per-key scales into an 8-slot ring.
+// Roles (576 threads):
+//   warp 0      producer (one thread): TMA of the two 64-row key boxes (a box
+//               never crosses a 64-token page) into a 6-stage ring, and of the
+//               group's queries (N x 128 B) into a double buffer.
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
-//               into one of two TMEM accumulators (2 x N columns).
-//   warps 2-9   epilogue: tcgen05.ld of the accumulator (lane = key), ReLU,
-//               head-weighted sum with w', times k_scale, coalesced fp32 store.
+//               into one of four (N <= 128) or two TMEM accumulators.
+//   warps 2-17  epilogue in 16/(4*NQ) sets that take alternate tiles (one
+//               set's TMEM-load latency overlaps another's math): tcgen05.ld
+//               of the accumulator (lane = key), ReLU, head-weighted sum with w'
+//               (packed fp32x2 FMAs), times the key's scale, coalesced store.
 // The L x H_I per-head score tensor lives only in TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -37,31 +38,36 @@ namespace {
 constexpr int kTileKeys = 128;
 constexpr int kDI = 128;
 constexpr int kHI = 64;
-constexpr int kStages = 6;
-constexpr int kScaleSlots = 8;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 2048;
 constexpr int kMaxCtaTiles = 512;
 constexpr int kKeyTileBytes = kTileKeys * kDI;   // 16 KB
 
+// Key-tile stages in flight: as many as shared memory allows beside the queries.
+template <int NQ>
+constexpr int num_stages() { return NQ <= 2 ? 10 : 6; }
+
+// TMEM accumulators per CTA: four of N columns when they fit in 512, else two.
+template <int NQ>
+constexpr int num_acc() { return NQ * kHI <= 128 ? 4 : 2; }
+
 template <int NQ>
 struct __align__(1024) IdxSmem {
-  uint8_t keys[kStages][kKeyTileBytes];
+  uint8_t keys[num_stages<NQ>()][kKeyTileBytes];
   uint8_t q[2][NQ * kHI * kDI];
-  float scales[kScaleSlots][kTileKeys];
-  float wq[kEpiWarps][(NQ >= 2 ? NQ / 2 : 1) * kHI];   // per epilogue warp: w' of its queries
+  float wq[kEpiWarps][kHI];                             // per epilogue warp: w' of its heads
   int32_t tile_row[kMaxCtaTiles][2];                    // physical row of each 64-key half, -1: none
   int32_t tile_off[kMaxGroups + 1];
   int32_t scan_tmp[kThreads / 32];
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[num_stages<NQ>()], empty[num_stages<NQ>()];
   uint64_t q_full[2], q_empty[2];
-  uint64_t acc_full[2], acc_empty[2];
-  uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
+  uint64_t acc_full[4], acc_empty[4];
   uint32_t tmem_base;
 };
 
 struct TcArgs {
+  long long* trace;           // profiling stamps (CTA 0, first 32 tiles) or null
   int num_rows, n_groups;
   const int32_t* row_seq;
   const int32_t* row_klen;
@@ -101,6 +107,23 @@ struct TileIter {
   }
 };
 
+__device__ __forceinline__ void istamp(long long* tr, int ev, int j) {
+  if (tr != nullptr && blockIdx.x == 0 && j < kTraceBlocks) tr[ev * kTraceBlocks + j] = clock64();
+}
+
+// ReLU of two fp32 bit patterns, packed low | high << 32 for an f32x2 operation.
+__device__ __forceinline__ unsigned long long relu2(uint32_t a, uint32_t b) {
+  return (unsigned long long)__float_as_uint(fmaxf(__uint_as_float(a), 0.f)) |
+         ((unsigned long long)__float_as_uint(fmaxf(__uint_as_float(b), 0.f)) << 32);
+}
+// d = a * b + c on two fp32 lanes at once (fma.rn.f32x2).
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 template <int NQ>
 __device__ __forceinline__ int group_max_klen(const TcArgs& a, int g) {
   int mk = 0;
@@ -118,6 +141,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                   TcArgs a) {
   constexpr int N = NQ * kHI;
   constexpr int kQBytes = N * kDI;
+  constexpr int kAcc = num_acc<NQ>();
+  constexpr int kStages = num_stages<NQ>();
   extern __shared__ __align__(1024) uint8_t smraw[];
   IdxSmem<NQ>& S = *reinterpret_cast<IdxSmem<NQ>*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -161,18 +186,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
-      mbar_init(&S.acc_full[i], 1);
-      mbar_init(&S.acc_empty[i], kEpiWarps);
     }
-    for (int i = 0; i < kScaleSlots; ++i) {
-      mbar_init(&S.sc_full[i], 32);          // one cp.async arrival per producer lane
-      mbar_init(&S.sc_empty[i], kEpiWarps);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&S.acc_full[i], 1);
+      mbar_init(&S.acc_empty[i], 4 * NQ);     // the warps of one epilogue set
     }
     fence_mbar_init();
   }
   __syncwarp();
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, 2 * N);
+    tmem_alloc(&S.tmem_base, kAcc * N);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -206,54 +229,41 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const bool run = ntile > 0 && ntile <= kMaxCtaTiles;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer warp
-    if (run) {
-      if (lane == 0) { prefetch_tmap(&tm_k); prefetch_tmap(&tm_q); }
+    // ------------------------------------------------------------ producer (lane 0): TMA only
+    if (run && lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_q);
       TileIter it;
       it.start(S.tile_off, a.n_groups, t_begin);
       int qcount = 0, j = 0;
       bool alive = true;
-      for (; j < ntile; ++j, it.next()) {
-        const int st = j % kStages, sl = j % kScaleSlots;
-        if (lane == 0) {
-          if (j == 0 || it.kt == 0) {
-            const int qb = qcount & 1;
-            alive = mbar_wait(&S.q_empty[qb], ((qcount >> 1) & 1) ^ 1, a.status, 1);
-            if (alive) {
-              mbar_expect_tx(&S.q_full[qb], kQBytes);
-              tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, it.g * NQ * kHI);
-            }
-          }
-          alive = alive && mbar_wait(&S.empty[st], ((j / kStages) & 1) ^ 1, a.status, 2);
-          if (alive) {
-            const int r0 = S.tile_row[j][0], r1 = S.tile_row[j][1];
-            const uint32_t bytes = (r0 >= 0 ? kKeyTileBytes / 2 : 0) + (r1 >= 0 ? kKeyTileBytes / 2 : 0);
-            if (bytes == 0) {
-              mbar_arrive(&S.full[st]);
-            } else {
-              mbar_expect_tx(&S.full[st], bytes);
-              if (r0 >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, r0);
-              if (r1 >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, r1);
-            }
-          }
-          alive = alive && mbar_wait(&S.sc_empty[sl], ((j / kScaleSlots) & 1) ^ 1, a.status, 9);
+      for (; j < ntile && alive; ++j, it.next()) {
+        const int st = j % kStages;
+        if (j == 0 || it.kt == 0) {
+          const int qb = qcount & 1;
+          alive = mbar_wait(&S.q_empty[qb], ((qcount >> 1) & 1) ^ 1, a.status, 1);
+          if (!alive) break;
+          mbar_expect_tx(&S.q_full[qb], kQBytes);
+          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, it.g * NQ * kHI);
+          ++qcount;
         }
-        if (j == 0 || it.kt == 0) ++qcount;
-        alive = __shfl_sync(0xffffffffu, alive, 0);
+        alive = mbar_wait(&S.empty[st], ((j / kStages) & 1) ^ 1, a.status, 2);
         if (!alive) break;
-        // the tile's 128 key scales: 4 per lane, asynchronously
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int k = i * 32 + lane;
-          const int r = S.tile_row[j][k >> 6];
-          if (r >= 0 && (int64_t)r + (k & 63) < a.map.num_tokens)
-            cp_async_4(&S.scales[sl][k], a.k_scale + (int64_t)r + (k & 63));
+        istamp(a.trace, 0, j);
+        const int r0 = S.tile_row[j][0], r1 = S.tile_row[j][1];
+        const uint32_t bytes = (r0 >= 0 ? kKeyTileBytes / 2 : 0) + (r1 >= 0 ? kKeyTileBytes / 2 : 0);
+        if (bytes == 0) {
+          mbar_arrive(&S.full[st]);
+        } else {
+          mbar_expect_tx(&S.full[st], bytes);
+          if (r0 >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, r0);
+          if (r1 >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, r1);
         }
-        cp_async_mbar_arrive(&S.sc_full[sl]);
+        istamp(a.trace, 1, j);
       }
       // tail: wait until the MMAs have released every stage and query buffer in
       // use, so no commit is still in flight to this CTA's shared memory at exit
-      if (alive && lane == 0) {
+      if (alive) {
         for (int st = 0; st < kStages && st < j; ++st) {
           const int last_use = (j - 1 - st) / kStages;
           if (!mbar_wait(&S.empty[st], last_use & 1, a.status, 7)) break;
@@ -263,7 +273,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           if (!mbar_wait(&S.q_empty[qb], last_use & 1, a.status, 8)) break;
         }
       }
-      cp_async_wait<0>();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -278,10 +287,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           ++qcount;
           if (!mbar_wait(&S.q_full[qcount & 1], (qcount >> 1) & 1, a.status, 3)) break;
         }
-        const int st = j % kStages, ab = j & 1;
+        const int st = j % kStages, ab = j % kAcc;
         if (!mbar_wait(&S.full[st], (j / kStages) & 1, a.status, 4)) break;
-        if (!mbar_wait(&S.acc_empty[ab], ((j >> 1) & 1) ^ 1, a.status, 5)) break;
+        if (!mbar_wait(&S.acc_empty[ab], ((j / kAcc) & 1) ^ 1, a.status, 5)) break;
         tc_fence_after();
+        istamp(a.trace, 2, j);
         const uint32_t ka = smem_u32(S.keys[st]);
         const uint32_t qa = smem_u32(S.q[qcount & 1]);
 #pragma unroll
@@ -290,93 +300,92 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                  idesc, k > 0);
         mma_commit(&S.empty[st]);
         mma_commit(&S.acc_full[ab]);
+        istamp(a.trace, 3, j);
         const bool last = (it.kt + 1 == it.ntiles) || (j + 1 == ntile);
         if (last) mma_commit(&S.q_empty[qcount & 1]);
         it.next();
       }
     }
   } else if (run) {
-    // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;               // 0..7
+    // ------------------------------------------------------------ epilogue (16 warps)
+    // The 16 warps form NSET = 16 / (4*NQ) sets of 4*NQ warps; set k takes the
+    // tiles j = k (mod NSET), so the sets sit in different phases and one set's
+    // TMEM-load latency overlaps another's arithmetic.  Warp (lq, qi) of a set
+    // reduces the 64 heads of query qi for keys 32lq..32lq+31 of its tiles.
+    // A wait that times out only marks the warp dead.
+    constexpr int WPS = 4 * NQ;
+    constexpr int NSET = kEpiWarps / WPS;
+    const int e = warp - 2;               // 0..15
+    const int set = e / WPS, wi = e % WPS;
     const int lq = warp & 3;              // TMEM lane quarter this warp may access
-    const int half = e >> 2;
+    const int qi = wi >> 2;
     const int row_in_tile = lq * 32 + lane;
-    constexpr int QPW = NQ >= 2 ? NQ / 2 : 1;   // queries this warp reduces
-    const bool active = NQ >= 2 || half == 0;
+    const uint32_t lane_off = (uint32_t)(lq * 32) << 16;
     TileIter it;
     it.start(S.tile_off, a.n_groups, t_begin);
-    int klen[QPW];
-    for (int j = 0; j < ntile; ++j, it.next()) {
-      if (j == 0 || it.kt == 0) {
-        for (int i = 0; i < QPW; ++i) {
-          const int r = it.g * NQ + half * QPW + i;
-          klen[i] = (active && r < a.num_rows) ? a.row_klen[r] : 0;
-        }
-        // w' = w * q_scale of this warp's queries into this warp's own slice
-        // (written and read by the same warp: __syncwarp orders it)
+    for (int k = 0; k < set && k < ntile; ++k) it.next();
+    int klen = 0, cur_g = -1;
+    bool dead = false;
+    for (int j = set; j < ntile; j += NSET) {
+      if (it.g != cur_g) {
+        cur_g = it.g;
+        const int r = it.g * NQ + qi;
+        klen = r < a.num_rows ? a.row_klen[r] : 0;
+        // w' = w * q_scale of this warp's query into its own slice
         __syncwarp();
-        for (int i = lane; i < QPW * kHI; i += 32) {
-          const int r = it.g * NQ + half * QPW + i / kHI, h = i % kHI;
-          float v = 0.f;
-          if (active && r < a.num_rows)
-            v = a.w[(int64_t)r * kHI + h] * a.q_scale[(int64_t)r * kHI + h];
-          S.wq[e][i] = v;
-        }
+        for (int q = lane; q < kHI; q += 32)
+          S.wq[e][q] = r < a.num_rows ? a.w[(int64_t)r * kHI + q] * a.q_scale[(int64_t)r * kHI + q] : 0.f;
         __syncwarp();
       }
-      const int ab = j & 1, sl = j % kScaleSlots;
-      if (!mbar_wait(&S.acc_full[ab], (j >> 1) & 1, a.status, 6)) break;
+      // key scale of this thread's key, loaded before the accumulator wait
+      float ks = 0.f;
+      {
+        const int rr = S.tile_row[j][row_in_tile >> 6];
+        const int64_t pr = (int64_t)rr + (row_in_tile & 63);
+        if (rr >= 0 && pr < a.map.num_tokens) ks = __ldg(a.k_scale + pr);
+      }
+      const int ab = j % kAcc;
+      dead = dead || !mbar_wait(&S.acc_full[ab], (j / kAcc) & 1, a.status, 6);
       tc_fence_after();
-      const int s = it.kt * kTileKeys + row_in_tile;
-      float res[QPW];
-      if (active) {
-#pragma unroll
-        for (int i = 0; i < QPW; ++i) {
-          const int qi = half * QPW + i;
-          const uint32_t col = tmem + ab * N + qi * kHI + ((uint32_t)(lq * 32) << 16);
-          uint32_t v0[32], v1[32];
-          tmem_ld32(col, v0);
-          tmem_ld32(col + 32, v1);
-          tmem_wait_ld();
-          const float4* wv = reinterpret_cast<const float4*>(&S.wq[e][i * kHI]);
-          float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-          for (int h = 0; h < 32; h += 4) {
-            const float4 w0 = wv[h / 4];
-            acc0 = fmaf(fmaxf(__uint_as_float(v0[h + 0]), 0.f), w0.x, acc0);
-            acc1 = fmaf(fmaxf(__uint_as_float(v0[h + 1]), 0.f), w0.y, acc1);
-            acc2 = fmaf(fmaxf(__uint_as_float(v0[h + 2]), 0.f), w0.z, acc2);
-            acc3 = fmaf(fmaxf(__uint_as_float(v0[h + 3]), 0.f), w0.w, acc3);
-            const float4 w1 = wv[8 + h / 4];
-            acc0 = fmaf(fmaxf(__uint_as_float(v1[h + 0]), 0.f), w1.x, acc0);
-            acc1 = fmaf(fmaxf(__uint_as_float(v1[h + 1]), 0.f), w1.y, acc1);
-            acc2 = fmaf(fmaxf(__uint_as_float(v1[h + 2]), 0.f), w1.z, acc2);
-            acc3 = fmaf(fmaxf(__uint_as_float(v1[h + 3]), 0.f), w1.w, acc3);
-          }
-          res[i] = (acc0 + acc1) + (acc2 + acc3);
-        }
-      }
+      if (threadIdx.x == 64) istamp(a.trace, 4, j);
+      const uint32_t col = tmem + lane_off + ab * N + qi * kHI;
+      uint32_t v0[32], v1[32];
+      tmem_ld32(col, v0);
+      tmem_ld32(col + 32, v1);
+      tmem_wait_ld_regs(v0);
+      tmem_wait_ld_regs(v1);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.acc_empty[ab]);
-      if (!mbar_wait(&S.sc_full[sl], (j / kScaleSlots) & 1, a.status, 10)) break;
-      const float ks = S.scales[sl][row_in_tile];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.sc_empty[sl]);
-      if (active) {
+      if (lane == 0) mbar_arrive(&S.acc_empty[ab]);      // values are in registers
+      // sum_h w'_h ReLU(x_h), two heads per packed fp32x2 FMA
+      const ulonglong2* wv = reinterpret_cast<const ulonglong2*>(&S.wq[e][0]);
+      unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int i = 0; i < QPW; ++i) {
-          const int r = it.g * NQ + half * QPW + i;
-          if (s < klen[i]) a.scores[(int64_t)r * a.ld + s] = res[i] * ks;
-        }
+      for (int h = 0; h < 32; h += 4) {
+        const ulonglong2 w0 = wv[h / 4], w1 = wv[8 + h / 4];
+        acc[0] = ffma2(relu2(v0[h + 0], v0[h + 1]), w0.x, acc[0]);
+        acc[1] = ffma2(relu2(v0[h + 2], v0[h + 3]), w0.y, acc[1]);
+        acc[2] = ffma2(relu2(v1[h + 0], v1[h + 1]), w1.x, acc[2]);
+        acc[3] = ffma2(relu2(v1[h + 2], v1[h + 3]), w1.y, acc[3]);
       }
+      float lo[4], hi[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        lo[q] = __uint_as_float((uint32_t)acc[q]);
+        hi[q] = __uint_as_float((uint32_t)(acc[q] >> 32));
+      }
+      const float sum = ((lo[0] + hi[0]) + (lo[1] + hi[1])) + ((lo[2] + hi[2]) + (lo[3] + hi[3]));
+      const int s = it.kt * kTileKeys + row_in_tile;
+      if (!dead && s < klen) a.scores[(int64_t)(it.g * NQ + qi) * a.ld + s] = sum * ks;
+      if (threadIdx.x == 64) istamp(a.trace, 7, j);
+      for (int k = 0; k < NSET; ++k) it.next();
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * N);
+    tmem_dealloc(tmem, kAcc * N);
   }
 }
 
@@ -450,6 +459,7 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     t.scores = a.scores + (int64_t)r0 * a.ld_scores;
     t.ld = a.ld_scores;
     t.status = a.status;
+    t.trace = trace_buffer();
     CUtensorMap tq;
     if (!make_tmap_rows128(&tq, static_cast<const uint8_t*>(a.q_idx) + (int64_t)r0 * kHI * kDI,
                            (uint64_t)t.num_rows * kHI, NQ * kHI)) {

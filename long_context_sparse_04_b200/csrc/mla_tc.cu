@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kH = 128, kDC = 512, kDR = 64, kD = kDC + kDR;
 constexpr int kBlk = 64;
-constexpr int kNS = 2;
+constexpr int kNS = 3;
 constexpr int kMaxKeys = 2048;
 constexpr int kThreads = 32 * 13;
 constexpr int kPieces = 36;                 // 16-byte pieces of one key's 288 dims per CTA
@@ -43,15 +43,21 @@ constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;
-constexpr uint32_t kXBytes = kH * 64 * sizeof(float);   // one exchanged logit tile
+// One exchanged tile of partial logits of 128 heads x 64 keys in the transport
+// format below (row max + 16-bit fixed-point distance to it).
+struct __align__(16) XTile {
+  uint4 d[kH * 8];                          // 8 x 16-byte pieces per head, swizzled
+  float m[kH];
+};
+constexpr uint32_t kXBytes = sizeof(XTile);
 
 struct __align__(1024) MlaSmem {
   uint8_t q[4][kH * 128];                   // Q latent dims of this CTA: 4 SW128 chunks of 64 dims
   uint8_t kv[kNS][4][kBlk * 128];           // gathered latent dims: 4 SW128 chunks x 64 keys
   uint8_t kv_rope[kNS][kBlk * 64];          // gathered RoPE dims (32), SW64
   uint8_t q_rope[kH * 64];                  // Q RoPE dims (32), SW64
-  float xbuf[kH * 64];                      // the peer's partial logits, 16-byte pieces swizzled
-  float sbuf[kH * 64];                      // this CTA's partial logits, bulk-copied to the peer
+  XTile xbuf;                               // the peer's partial logits of the current block
+  XTile sbuf;                               // this CTA's partial logits, bulk-copied to the peer
   int32_t rows[kMaxKeys];                   // physical cache row per selected key, -1 = none
   unsigned long long valid[kMaxKeys / kBlk];
   uint64_t q_full, x_full, x_free;
@@ -70,6 +76,36 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Transport format of a partial logit row (log2 domain) between the two CTAs:
+// the row max m (fp32) and, per key, u = round(1024 * (m - z)) as a 16-bit
+// integer saturated at 65535 (a key 64 below the row max carries a weight under
+// 2^-64).  Error <= 2^-11 in the exponent (0.034% in the weight).  Encoding and
+// decoding use a float magic-number add, so no conversion instruction is needed.
+constexpr float kFix = 1024.f, kFixInv = 1.f / 1024.f, kMagic = 12582912.f;   // 1.5 * 2^23
+__device__ __forceinline__ float encode_partial(float (&z)[64], float c, uint32_t (&pk)[32]) {
+  float pm[8];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    z[i] *= c;
+    pm[i & 7] = (i < 8) ? z[i] : fmaxf(pm[i & 7], z[i]);
+  }
+  const float m = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                        fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t u0 = __float_as_uint(fminf((m - z[2 * i]) * kFix, 65535.f) + kMagic);
+    const uint32_t u1 = __float_as_uint(fminf((m - z[2 * i + 1]) * kFix, 65535.f) + kMagic);
+    pk[i] = __byte_perm(u0, u1, 0x5410);          // low 16 bits of each
+  }
+  return m;
+}
+// z of the two keys packed in w, given the row max m.
+__device__ __forceinline__ float2 decode_partial(uint32_t w, float m) {
+  const float u0 = __uint_as_float(0x4B000000u | (w & 0xFFFFu)) - 8388608.f;
+  const float u1 = __uint_as_float(0x4B000000u | (w >> 16)) - 8388608.f;
+  return make_float2(fmaf(-u0, kFixInv, m), fmaf(-u1, kFixInv, m));
 }
 
 __device__ __forceinline__ void tstamp(long long* tr, uint32_t rank, int ev, int j) {
@@ -157,7 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       for (int j = 0; j < nblk; ++j) {
         const int st = j % kNS;
         if (!mbar_wait(&S.kv_empty[st], ((j / kNS) & 1) ^ 1, a.status, 21)) { alive = false; break; }
-        if (tid == 0) tstamp(a.trace, rank, 0, j);
         for (int i = 0; i < (kBlk * kPieces) / 128; ++i) {
           const int qi = i * 128 + tid;
           const int key = qi / kPieces, c = qi - key * kPieces;
@@ -182,33 +217,36 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     // times out only marks the warpgroup dead: the named barriers stay uniform.
     const int h = threadIdx.x - 128;                          // head = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const float c = a.sm_scale * kLog2e;
     bool dead = false;
     for (int j = 0; j < nblk; ++j) {
       const int b = j & 1;
-      uint32_t v[64];
+      float z[64];
+      uint32_t pk[32];
+      float m = 0.f;
       dead = dead || !mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 22);
       if (!dead) {
         tc_fence_after();
-        tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&z[0]));
+        tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&z[32]));
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&S.s_free[b]);
+        m = encode_partial(z, c, pk);
       }
       if (h == 0 && j > 0) bulk_wait_read0();               // the previous copy has left sbuf
       named_bar_sync(2, 128);
       if (!dead) {
 #pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4)
-          *reinterpret_cast<uint4*>(&S.sbuf[h * 64 + 4 * (q4 ^ (h & 15))]) =
-              make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        for (int q = 0; q < 8; ++q)
+          S.sbuf.d[h * 8 + (q ^ (h & 7))] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        S.sbuf.m[h] = m;
       }
       fence_proxy_async_smem();                              // sbuf writes -> async copy engine
       named_bar_sync(2, 128);
       if (h == 0 && !dead) {
         if (mbar_wait_cluster(&S.x_free, (j & 1) ^ 1, a.status, 23)) {
-          tstamp(a.trace, rank, 7, j);
-          bulk_copy_to_peer(S.xbuf, S.sbuf, kXBytes, &S.x_full, peer);
+          bulk_copy_to_peer(&S.xbuf, &S.sbuf, kXBytes, &S.x_full, peer);
           bulk_commit();
         }
       }
@@ -234,22 +272,34 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&S.s_free[b]);
-      // the peer's partial logits of this block, then S = own + peer (same bits in both CTAs)
+      // z = c * S_own (exact) + the peer's partial (decoded).  The two
+      // CTAs see the same sum up to that rounding; each keeps its own softmax
+      // state (m, l), used for its own half of the value dims.
+#pragma unroll
+      for (int i = 0; i < 64; ++i) s[i] *= c;
       dead = dead || !mbar_wait_cluster(&S.x_full, j & 1, a.status, 24);
       if (h == 0) tstamp(a.trace, rank, 5, j);
+      const float m_peer = S.xbuf.m[h];
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4) {
-        const float4 o = *reinterpret_cast<const float4*>(&S.xbuf[h * 64 + 4 * (q4 ^ (h & 15))]);
-        s[4 * q4 + 0] += o.x;
-        s[4 * q4 + 1] += o.y;
-        s[4 * q4 + 2] += o.z;
-        s[4 * q4 + 3] += o.w;
+      for (int q = 0; q < 8; ++q) {
+        const uint4 w4 = S.xbuf.d[h * 8 + (q ^ (h & 7))];
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = decode_partial(w[e], m_peer);
+          s[8 * q + 2 * e] += f.x;
+          s[8 * q + 2 * e + 1] += f.y;
+        }
       }
+      if (h == 0) tstamp(a.trace, rank, 0, j);
       if (named_bar_or(3, 128, dead)) { dead = true; break; }   // whole tile read, all alive
       if (h == 0) {
         if (j + 1 < nblk) mbar_expect_tx(&S.x_full, kXBytes);   // arm the next transfer first
-        mbar_arrive_cluster(&S.x_free, peer);                    // then free the buffer
+        // then free the buffer: every thread's reads of it were consumed before
+        // the barrier above, so the arrive needs no release ordering
+        mbar_arrive_cluster_relaxed(&S.x_free, peer);
       }
+      if (h == 0) tstamp(a.trace, rank, 1, j);
       // masked (only partial blocks), scaled logits in the log2 domain; block max
       const unsigned long long mask = S.valid[j];
       if (mask != ~0ull) {
@@ -259,12 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       }
       float pm[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) pm[i] = s[i] * c;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] *= c;
-        if (i >= 8) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
-      }
+      for (int i = 0; i < 64; ++i) pm[i & 7] = (i < 8) ? s[i] : fmaxf(pm[i & 7], s[i]);
       const float mb = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                              fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       // lazy rescale (warp-uniform because tcgen05.ld/st are warp-collective)
@@ -302,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         p2[i] = pack_bf16x2(p0, p1);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      if (h == 0) tstamp(a.trace, rank, 7, j);
       // P buffer b is free once the PV of block j-2 is done
       dead = dead || !mbar_wait(&S.pv_done[b], ((j >> 1) & 1) ^ 1, a.status, 26);
       tc_fence_after();
@@ -347,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         }
       }
     }
-    if (rank == 0) {
+    if (a.splits > 1 || rank == 0) {
       if (a.splits > 1) {
-        reinterpret_cast<float2*>(a.part_ml)[((int64_t)t * a.splits + sp) * kH + h] =
+        reinterpret_cast<float2*>(a.part_ml)[(((int64_t)t * a.splits + sp) * 2 + rank) * kH + h] =
             make_float2(m_used, l);
       } else if (a.lse) {
         a.lse[ro] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
@@ -368,7 +414,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
           const int st = j % kNS, b = j & 1;
           if (!(ok = mbar_wait(&S.kv_full[st], (j / kNS) & 1, a.status, 32))) break;
           fence_proxy_async_smem();           // gathered (generic-proxy) writes -> tensor cores
-          tstamp(a.trace, rank, 1, j);
           if (!(ok = mbar_wait(&S.s_free[b], ((j >> 1) & 1) ^ 1, a.status, 33))) break;
           tc_fence_after();
           const uint32_t ka = smem_u32(S.kv[st][0]), kra = smem_u32(S.kv_rope[st]);
@@ -414,16 +459,20 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
 
 // out[t,h,:] = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max_s m_s); fixed split order.
 __global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
+  // thread i: value dims 4i..4i+3, produced by CTA rank (4i >= 256) with that
+  // CTA's own softmax state (m, l) of each split
   trace_kernel(a.status, DSA_KERNEL_MLA_COMBINE);
   const int th = blockIdx.x;
   const int t = th / kH, h = th % kH;
+  const int r = threadIdx.x >= 64 ? 1 : 0;
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
+  auto at = [&](int s) { return ml[(((int64_t)t * a.splits + s) * 2 + r) * kH + h]; };
   float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, ml[((int64_t)t * a.splits + s) * kH + h].x);
+  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, at(s).x);
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < a.splits; ++s) {
-    const float2 v = ml[((int64_t)t * a.splits + s) * kH + h];
+    const float2 v = at(s);
     const float w = (v.x == -INFINITY) ? 0.f : exp2f(v.x - M);
     L += w * v.y;
     const float4 o = reinterpret_cast<const float4*>(
@@ -467,7 +516,7 @@ int mla_tc_splits(int num_rows) {
 
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits) {
   if (splits <= 1) return 0;
-  return (size_t)num_rows * splits * n_heads * (d_c * sizeof(float) + 2 * sizeof(float));
+  return (size_t)num_rows * splits * n_heads * (d_c * sizeof(float) + 4 * sizeof(float));
 }
 
 dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
