@@ -376,6 +376,7 @@ dsa_status dsa_topk(const dsa_dims* dims, const dsa_rows* rows, const float* sco
   a.topk = dims->topk;
   a.idx = idx;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
+  a.trace = trace_buffer();
   return launch_topk(a, rows->max_klen, (cudaStream_t)stream);
 }
 
@@ -428,6 +429,7 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   ta.topk = dims->topk;
   ta.idx = idx;
   ta.status = reinterpret_cast<DeviceStatus*>(ws);
+  ta.trace = trace_buffer();
   if ((st = launch_topk(ta, rows->max_klen, s))) return st;
   stage_event(2, s);
   MlaArgs ma = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
@@ -483,6 +485,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     ta.topk = dims->topk;
     ta.idx = idx;
     ta.status = reinterpret_cast<DeviceStatus*>(ws);
+  ta.trace = trace_buffer();
     if ((st = launch_topk(ta, rows->max_klen, s))) return st;
     MlaArgs ma = mla_args(dims, &cr, cache, qq, idx, oo, ll, ws, p);
     if ((st = run_mla(dims, ma, s))) return st;

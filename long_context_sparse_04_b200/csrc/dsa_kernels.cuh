@@ -32,6 +32,7 @@ struct TopkArgs {
   int topk;
   int32_t* idx;               // [T, topk]
   DeviceStatus* status;
+  long long* trace;           // profiling stamps or null
 };
 
 struct MlaArgs {
