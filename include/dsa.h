@@ -25,7 +25,8 @@
  *  - All pointers except the dsa_* descriptor structs are DEVICE pointers owned
  *    by the caller.  The library allocates no device memory: scratch comes from
  *    the caller's workspace `ws` (size from dsa_workspace_size, 256-byte
- *    aligned).  Descriptor structs are read on the host during the call only.
+ *    aligned), or for dsa_sparse_mla_fwd_noalloc from a static array inside
+ *    the library.  Descriptor structs are read on the host during the call only.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream).  No entry point synchronises, except
  *    dsa_read_device_status.
@@ -213,6 +214,30 @@ dsa_status dsa_topk(const dsa_dims* dims, const dsa_rows* rows, const float* sco
 dsa_status dsa_sparse_mla_fwd(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
                               const void* q, const int32_t* idx, void* out, float* lse,
                               void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* dsa_sparse_mla_fwd without a caller workspace, for callers that cannot hand
+ * out device memory.  The sparse attention pages have no counterpart of this
+ * call: it is a deployment convenience.  Arguments, layouts and results are
+ * those of dsa_sparse_mla_fwd, bit for bit (same kernels, same split plan).
+ * Scratch: a file-scope static device array of 20 MiB (256-byte status block
+ * + split-K partials) inside the library.  Nothing is allocated: no
+ * cudaMalloc/cudaFree, no allocating library routine.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture.  Later calls may be captured.
+ *   - Each call clears the status block (cudaMemsetAsync on `stream`); the
+ *     partials need no clearing, every split writes its own.  Device-side
+ *     range errors are recorded there but cannot be read back through this
+ *     call: use dsa_sparse_mla_fwd with a workspace for checked runs.
+ *   - Every call on a device shares the one array, so calls that overlap
+ *     (different streams, or host threads racing on one device) race on it
+ *     and corrupt each other's partials.  Serialise them.
+ * Returns DSA_ERR_WORKSPACE, with the sizes in dsa_last_error(), when the
+ * split plan needs more than the 20 MiB (more rows x splits than the array
+ * holds), and the argument errors of dsa_sparse_mla_fwd. */
+dsa_status dsa_sparse_mla_fwd_noalloc(const dsa_dims* dims, const dsa_rows* rows,
+                                      const dsa_cache* cache, const void* q, const int32_t* idx,
+                                      void* out, float* lse, dsa_stream_t stream);
 
 /* The three stages for a batch of decode rows (few rows per sequence), one
  * enqueue, no host synchronisation.  Scores and indices live in ws unless

@@ -55,6 +55,7 @@ _SIGS = {
                                           ctypes.c_size_t, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P]),
     "dsa_sparse_mla_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "dsa_sparse_mla_fwd_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "dsa_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.c_size_t, _P]),
     "dsa_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -138,6 +139,11 @@ def dsa_topk(dims, rows, scores, ld_scores, idx, ws, ws_bytes, stream, check=Tru
 def dsa_sparse_mla_fwd(dims, rows, cache, q, idx, out, lse, ws, ws_bytes, stream, check=True):
     return _call("dsa_sparse_mla_fwd", _ref(dims), _ref(rows), _ref(cache), q, idx, out, lse,
                  ws, ws_bytes, stream, check=check)
+
+
+def dsa_sparse_mla_fwd_noalloc(dims, rows, cache, q, idx, out, lse, stream, check=True):
+    return _call("dsa_sparse_mla_fwd_noalloc", _ref(dims), _ref(rows), _ref(cache), q, idx, out,
+                 lse, stream, check=check)
 
 
 def dsa_decode_step(dims, rows, cache, q_idx, q_scale, w, q, out, lse, dbg_scores, dbg_idx,

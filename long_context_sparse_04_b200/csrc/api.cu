@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "dsa_kernels.cuh"
 
@@ -234,6 +235,39 @@ dsa_status run_mla(const dsa_dims* d, MlaArgs& a, cudaStream_t s) {
   return launch_mla_simt(a, s);
 }
 
+// Scratch of dsa_sparse_mla_fwd_noalloc: the 256-byte status block followed
+// by the split-K partials, laid out as the caller workspace of
+// dsa_sparse_mla_fwd.  20 MiB holds every split plan of the tensor-core path
+// (H = 128, d_c = 512) on a 148-SM device: one CTA pair per (row, split), so
+// rows * splits <= 74, 74 * 128 * 2064 bytes = 18.6 MiB.
+constexpr size_t kNoAllocScratchBytes = size_t(20) << 20;
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device and kept.
+dsa_status noalloc_scratch(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* ptr[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    set_error("no current CUDA device (or device index >= %d)", kMaxDevices);
+    return DSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      set_error("cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+      return DSA_ERR_CUDA;
+    }
+    ptr[dev] = p;
+  }
+  *out = ptr[dev];
+  return DSA_OK;
+}
+
 }  // namespace
 }  // namespace dsa
 
@@ -393,6 +427,33 @@ dsa_status dsa_sparse_mla_fwd(const dsa_dims* dims, const dsa_rows* rows, const 
   }
   const WsPlan p = plan(dims, rows, DSA_OP_SPARSE_MLA);
   if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  MlaArgs a = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
+  return run_mla(dims, a, (cudaStream_t)stream);
+}
+
+dsa_status dsa_sparse_mla_fwd_noalloc(const dsa_dims* dims, const dsa_rows* rows,
+                                      const dsa_cache* cache, const void* q, const int32_t* idx,
+                                      void* out, float* lse, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows)) ||
+      (st = check_cache(cache, dims, false, true)))
+    return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(q && idx && out, "q / idx / out is NULL");
+    CHECK_ARG(aligned(q, 16) && aligned(out, 16), "q and out must be 16-byte aligned");
+  }
+  const WsPlan p = plan(dims, rows, DSA_OP_SPARSE_MLA);
+  if (p.total > kNoAllocScratchBytes) {
+    set_error("sparse MLA of %d rows needs %zu bytes of scratch; the static scratch holds %zu",
+              rows->num_rows, p.total, kNoAllocScratchBytes);
+    return DSA_ERR_WORKSPACE;
+  }
+  void* ws = nullptr;
+  if ((st = noalloc_scratch(&ws))) return st;
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream) != cudaSuccess) {
+    set_error("clearing the status block failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return DSA_ERR_CUDA;
+  }
   MlaArgs a = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
   return run_mla(dims, a, (cudaStream_t)stream);
 }
