@@ -2,24 +2,33 @@
 // Attention DSA Architecture Guide", section "Stage 2: Fine-Grained Token
 // Selection and Output Computation", selection equation S_t = TopK(I[t,:], k)).
 //
-// One cluster of `csize` CTAs (1..8, 512 threads each) per query row.  Each CTA
-// copies a contiguous segment of the row into shared memory (cp.async, all
-// loads in flight at once) and turns it in place into order-preserving uint32
-// keys (float -> key, -0 mapped to +0).  The k-th largest key T is found digit
-// by digit (12 + 10 + 10 bits, most significant first):
-//   * every CTA builds a histogram of its keys that match the prefix so far;
-//   * the cluster merges them as a reduce-scatter: CTA r sums bins
-//     [r*B/csize, (r+1)*B/csize) over the cluster through distributed shared
-//     memory, the per-CTA slice totals are exchanged, and the CTA whose slice
-//     holds the k-th key finds the bin and tells the others;
-//   * after the first digit only the keys of the threshold bin can matter, so
-//     each CTA moves them to a candidate list and later digits scan the list.
-// The output pass walks the segment in position order (lane-interleaved, so
-// shared-memory loads are conflict free, with warp ballots for the ordering)
-// and keeps key > T, and key == T while the running count of equal keys
-// (across the cluster, in position order) is below the number still needed.
-// The selected positions come out sorted ascending with ties going to the
-// lower position, without a sort.  Rows with klen <= k return 0..klen-1 then -1.
+// One cluster of `csize` CTAs (1..8, 512 threads each) per query row.  CTA r
+// copies segment r of the row into shared memory (cp.async, all pieces in
+// flight at once) and turns it in place into order-preserving uint32 keys
+// (float -> key, -0 mapped to +0).  Full passes read four keys per thread.
+//
+// 1. Histogram of the top 12 key bits; the cluster merges the histograms
+//    (CTA r sums a slice of the bins over the cluster through distributed
+//    shared memory) and every CTA finds the bin B0 holding the k-th largest
+//    key, the rank `need0` of that key inside the bin, and the bin's size c0.
+// 2. Only keys in bin B0 or above can be selected (about k plus one bin per
+//    row, ~2% of the keys).  They are marked in a bitmap of the segment, one
+//    32-bit word per thread; every later pass visits set bits only.
+// 3. When c0 is small (the usual case) every CTA sends its keys of bin B0,
+//    and its count of keys above B0, to every CTA of the cluster; after one
+//    cluster barrier each CTA finishes the selection alone: two more 10-bit
+//    digits over the c0 gathered keys give the k-th largest key T and the
+//    number `need` of keys equal to T that are taken.  Otherwise the last two
+//    digits run as cluster-wide histograms like step 1.
+// 4. The output pass walks the marked keys in position order (thread w owns
+//    positions [32w, 32w+32); a block scan of the per-thread counts orders
+//    the threads) and keeps key > T, and key == T while the number of equal
+//    keys before it (across the cluster, in position order) is below `need`.
+//    The positions come out ascending with ties going to the lower position,
+//    without a sort.  A segment longer than the cache (rows past 8 * 16384
+//    keys) skips the bitmap and scans the segment instead, warp w owning a
+//    contiguous range and warp ballots giving the order inside it.
+// Rows with klen <= k return 0..klen-1 then -1.
 #include "dsa_kernels.cuh"
 
 namespace dsa {
@@ -29,27 +38,48 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins0 = 4096;       // first digit: bits 31..20
+constexpr int kBins = 1024;        // second and third digits: bits 19..10, 9..0
 constexpr int kCacheCap = 16384;   // keys of the segment kept in smem
-constexpr int kCandCap = 4096;     // candidates of the threshold bin per CTA
 constexpr int kMaxCluster = 8;
+constexpr int kGatherCap = 2048;   // threshold-bin keys of a row gathered in every CTA
+constexpr int kStampsPerCta = 16;
 
-__device__ __forceinline__ void kstamp(long long* tr, int ev) {
-  if (tr != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && ev < kTraceBlocks) tr[ev] = clock64();
+// clock64 stamps of the first cluster, [rank][event], when a trace buffer is set
+__device__ __forceinline__ void kstamp(long long* tr, uint32_t csize, uint32_t rank, int ev) {
+  if (tr != nullptr && blockIdx.x < csize && threadIdx.x == 0)
+    tr[rank * kStampsPerCta + ev] = clock64();
 }
 
 struct TopkSmem {
   uint32_t keys[kCacheCap];
   uint32_t hist[kBins0];
-  uint32_t cand_key[kCandCap];
-  uint32_t slice_tot[2][kMaxCluster];   // per-CTA slice totals, by digit parity
-  uint32_t counts[kMaxCluster][2];      // per-CTA (n_gt, n_eq)
+  uint32_t slice[kBins0 / 2];            // merged slice (csize >= 2); later a local histogram
+  uint32_t bits[kCacheCap / 32];         // keys in bin B0 or above
+  uint32_t gather[kGatherCap];           // keys of bin B0 of the whole row, by rank
+  uint32_t lhist[2][kBins];              // local histograms of the last two digits
+  uint32_t above[kMaxCluster];           // keys above bin B0, per rank
+  uint32_t slice_tot[kMaxCluster];       // slice totals of every CTA
+  uint32_t counts[kMaxCluster][2];       // (n_gt, n_eq) of every CTA (radix path)
   uint32_t warp_tmp[kWarps];
   uint32_t warp_cnt[kWarps][2];
-  uint32_t cand_n;
-  uint32_t sel[2][2];                   // (bin, need) found for digit d, by parity
+  uint32_t sel_bin, sel_need, sel_cnt;
+  uint32_t goff, gcount;
 };
 
-// Exclusive prefix over the block of one value per thread (512 threads).
+// Sum over the block (512 threads); every thread gets the total.
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = __reduce_add_sync(0xffffffffu, v);
+  if (lane == 0) tmp[warp] = v;
+  __syncthreads();
+  uint32_t all = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) all += tmp[w];
+  __syncthreads();
+  return all;
+}
+
+// Exclusive prefix over the block of one value per thread, in thread order.
 __device__ __forceinline__ uint32_t block_excl_prefix(uint32_t v, uint32_t* tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
@@ -68,87 +98,116 @@ __device__ __forceinline__ uint32_t block_excl_prefix(uint32_t v, uint32_t* tmp,
     all += s;
   }
   __syncthreads();
-  if (total) *total = all;
+  *total = all;
   return before + x - v;
 }
 
-// Shared histogram increment.  Row scores spread over many bins (a 32-key
-// warp round hits ~25 distinct bins), so warp-level aggregation of equal bins
-// buys nothing; the shared-memory atomic unit resolves the rare collisions.
-__device__ __forceinline__ void hist_add(uint32_t* hist, bool valid, uint32_t bin) {
-  if (valid) atomicAdd(&hist[bin], 1u);
-}
-
-// Cluster-wide selection of the bin holding the `need`-th largest key among
-// `nbins` histogram bins (S.hist of every CTA).  Returns (bin, need within bin)
-// in S.sel[par] of every CTA.  Two cluster barriers.
-__device__ void cluster_select(TopkSmem& S, int nbins, uint32_t need, uint32_t csize,
-                               uint32_t rank, int par) {
-  const int slice = nbins / (int)csize;              // bins owned by this CTA
-  const int b0 = (int)rank * slice;
-  cluster_sync();                                    // all histograms complete
-  // this CTA's slice, summed over the cluster: one bin per thread (slice <= 4096)
+// Among `nb` bins (higher bins hold larger keys) whose counts are at `bins` -
+// in CTA `owner`'s shared memory when `remote` - find the bin holding the
+// need-th largest key, given `above` keys in higher bins.  Sets S.sel_bin
+// (bin_base + bin), S.sel_need (rank inside the bin), S.sel_cnt (its count).
+__device__ void search_bins(TopkSmem& S, const uint32_t* bins, bool remote, uint32_t owner, int nb,
+                            int bin_base, uint32_t above, uint32_t need) {
+  const int tid = threadIdx.x;
+  const int per = (nb + kThreads - 1) / kThreads;   // 1..8
   uint32_t mine[8];
   uint32_t local = 0;
-  const int per = (slice + kThreads - 1) / kThreads; // 1..8 bins per thread
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
+    const int j = tid * per + i;
     mine[i] = 0;
-    if (i < per) {
-      const int b = b0 + threadIdx.x * per + i;
-      if (threadIdx.x * per + i < slice) {
-        if (csize == 1) {
-          mine[i] = S.hist[b];
-        } else {
-          uint32_t vv[kMaxCluster];
-#pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r)
-            vv[r] = r < (int)csize ? ld_dsmem_u32(mapa(&S.hist[b], (uint32_t)r)) : 0u;
-#pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r) mine[i] += vv[r];
-        }
-      }
-    }
+    if (i < per && j < nb) mine[i] = remote ? ld_dsmem_u32(mapa(&bins[j], owner)) : bins[j];
     local += mine[i];
   }
-  // suffix position of each thread's bins within the slice (bins descending = threads descending)
-  uint32_t total;
-  const uint32_t before = block_excl_prefix(local, S.warp_tmp, &total);
-  const uint32_t above_in_slice = total - before - local;   // keys in higher bins of the slice
-  // slice totals to every CTA
-  if (threadIdx.x == 0) {
-    for (uint32_t r = 0; r < csize; ++r) {
-      if (csize == 1) S.slice_tot[par][rank] = total;
-      else st_dsmem_u32(mapa(&S.slice_tot[par][rank], r), total);
-    }
-  }
-  cluster_sync();
-  // keys above this CTA's slice: all slices of higher rank
-  uint32_t above = 0;
-  for (uint32_t r = rank + 1; r < csize; ++r) above += S.slice_tot[par][r];
-  if (above < need && above + total >= need) {       // the slice holding the need-th key
-    uint32_t cum = above + above_in_slice;
+  uint32_t tot;
+  const uint32_t before = block_excl_prefix(local, S.warp_tmp, &tot);
+  uint32_t cum = above + (tot - before - local);      // keys in bins above this thread's
 #pragma unroll
-    for (int i = 7; i >= 0; --i) {
-      if (i < per) {
-        const uint32_t c = mine[i];
-        if (cum < need && cum + c >= need) {
-          const int b = b0 + threadIdx.x * per + i;
-          for (uint32_t r = 0; r < csize; ++r) {
-            if (csize == 1) {
-              S.sel[par][0] = (uint32_t)b;
-              S.sel[par][1] = need - cum;
-            } else {
-              st_dsmem_u32(mapa(&S.sel[par][0], r), (uint32_t)b);
-              st_dsmem_u32(mapa(&S.sel[par][1], r), need - cum);
-            }
-          }
-        }
-        cum += c;
+  for (int i = 7; i >= 0; --i) {
+    if (i < per) {
+      const uint32_t c = mine[i];
+      if (cum < need && cum + c >= need) {
+        S.sel_bin = (uint32_t)(bin_base + tid * per + i);
+        S.sel_need = need - cum;
+        S.sel_cnt = c;
       }
+      cum += c;
     }
   }
-  cluster_sync();                                    // (bin, need) everywhere
+  __syncthreads();
+}
+
+// Warp-level search of 1024 local bins: the bin holding the need-th largest
+// key, and the rank of that key inside it.  Lane L sums bins [32L, 32L+32)
+// (eight 16-byte loads in a lane-rotated order, so the eight lanes of each
+// load phase hit distinct banks); suffix sums over the lanes locate the lane
+// L* holding the key, then the warp reads L*'s 32 bins one per lane and a
+// second suffix scan locates the bin.
+__device__ __forceinline__ void warp_search_1024(const uint32_t* bins, uint32_t need,
+                                                 uint32_t* sel_bin, uint32_t* sel_need) {
+  const int lane = threadIdx.x & 31;
+  const uint4* mine = reinterpret_cast<const uint4*>(bins + 32 * lane);
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 x = mine[(i + lane) & 7];
+    s += x.x + x.y + x.z + x.w;
+  }
+  auto suffix = [&](uint32_t v) {                      // sum over lanes >= this one
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, v, off);
+      if (lane + off < 32) v += y;
+    }
+    return v;
+  };
+  const uint32_t above = suffix(s) - s;                // keys in the bins of higher lanes
+  const uint32_t hit = __ballot_sync(0xffffffffu, above < need && above + s >= need);
+  const int ls = __ffs(hit) - 1;                       // exactly one lane
+  const uint32_t base = __shfl_sync(0xffffffffu, above, ls);
+  const uint32_t c = bins[32 * ls + lane];
+  const uint32_t cum = base + suffix(c) - c;           // keys in higher bins
+  if (cum < need && cum + c >= need) {
+    *sel_bin = (uint32_t)(32 * ls + lane);
+    *sel_need = need - cum;
+  }
+}
+
+// The bin of the need-th largest key among `nbins` bins of S.hist summed over
+// the cluster (S.sel_* on every CTA).  Two cluster barriers.
+__device__ void cluster_select(TopkSmem& S, int nbins, uint32_t need, uint32_t csize,
+                               uint32_t rank) {
+  const int tid = threadIdx.x;
+  if (csize == 1) {
+    __syncthreads();                                  // the histogram is complete
+    search_bins(S, S.hist, false, 0, nbins, 0, 0, need);
+    return;
+  }
+  const int slice = nbins / (int)csize;
+  const int b0 = (int)rank * slice;
+  cluster_sync();                                     // every histogram is complete
+  uint32_t part = 0;
+  for (int j = tid; j < slice; j += kThreads) {
+    uint32_t vv[kMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r)
+      vv[r] = r < (int)csize ? ld_dsmem_u32(mapa(&S.hist[b0 + j], (uint32_t)r)) : 0u;
+    uint32_t c = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) c += vv[r];
+    S.slice[j] = c;
+    part += c;
+  }
+  const uint32_t total = block_sum(part, S.warp_tmp);
+  if (tid < (int)csize) st_dsmem_u32(mapa(&S.slice_tot[rank], (uint32_t)tid), total);
+  cluster_sync();                                     // slices and their totals published
+  uint32_t owner = 0, above = 0;                      // slices of higher rank hold higher bins
+  for (int r = (int)csize - 1; r >= 0; --r) {
+    const uint32_t tot = S.slice_tot[r];
+    if (above + tot >= need) { owner = (uint32_t)r; break; }
+    above += tot;
+  }
+  search_bins(S, S.slice, owner != rank, owner, slice, (int)owner * slice, above, need);
 }
 
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
@@ -163,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const int klen = a.row_klen[t];
   int32_t* out = a.idx + (int64_t)t * k;
 
-  kstamp(a.trace, 0);
+  kstamp(a.trace, csize, rank, 0);
   if (klen <= k) {  // uniform over the cluster; no DSMEM was touched
     for (int i = rank * kThreads + tid; i < k; i += csize * kThreads) out[i] = i < klen ? i : -1;
     return;
@@ -172,9 +231,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const float* row = a.scores + (int64_t)t * a.ld_scores;
   const int seg = (((klen + (int)csize - 1) / (int)csize) + 3) & ~3;
   const int lo = min((int)rank * seg, klen);
-  const int hi = min(lo + seg, klen);
-  const int n = hi - lo;
-  const int ncache = min(n, kCacheCap);
+  const int n = min(lo + seg, klen) - lo;
+  const int ncache = min(n, kCacheCap);     // n > kCacheCap only past 8 * 16384 keys
+  const int nvec = (n + 3) >> 2;
   const float* srow = row + lo;
 
   // ---- the segment into shared memory: every 16-byte piece in flight at once
@@ -185,160 +244,309 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       S.keys[i] = __float_as_uint(__ldcg(srow + i));
   }
   for (int i = tid; i < kBins0; i += kThreads) S.hist[i] = 0;
-  if (tid == 0) S.cand_n = 0;
   cp_async_wait_all();
   __syncthreads();
-  kstamp(a.trace, 1);
+  kstamp(a.trace, csize, rank, 1);
 
-  auto key_at = [&](int i) -> uint32_t {
-    return i < ncache ? S.keys[i] : float_key(__ldcg(srow + i));
-  };
-
-  // ---- digit 0: keys in place, histogram of bits 31..20
-  const int nround = (n + kThreads - 1) / kThreads;
-#pragma unroll 4
-  for (int r = 0; r < nround; ++r) {
-    const int i = r * kThreads + tid;
-    const bool v = i < n;
-    uint32_t key = 0;
-    if (v) {
-      if (i < ncache) {
-        key = float_key(__uint_as_float(S.keys[i]));
-        S.keys[i] = key;
-      } else {
-        key = float_key(__ldcg(srow + i));
-      }
-    }
-    hist_add(S.hist, v, key >> 20);
-  }
-  kstamp(a.trace, 2);
-  cluster_select(S, kBins0, (uint32_t)k, csize, rank, 0);
-  uint32_t prefix = S.sel[0][0];
-  uint32_t need = S.sel[0][1];
-  kstamp(a.trace, 3);
-
-  // ---- candidates of the threshold bin (warp-aggregated appends); this
-  // CTA's own histogram still says how many there are
-  const bool use_cand = S.hist[prefix] <= (uint32_t)kCandCap;
-  if (use_cand) {
-#pragma unroll 4
-    for (int r = 0; r < nround; ++r) {
-      const int i = r * kThreads + tid;
-      uint32_t key = 0;
-      const bool v = (i < n) && (((key = key_at(i)) >> 20) == prefix);
-      const uint32_t m = __ballot_sync(0xffffffffu, v);
-      uint32_t base = 0;
-      if (lane == 0 && m) base = atomicAdd(&S.cand_n, (uint32_t)__popc(m));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if (v) {
-        const uint32_t slot = base + __popc(m & ((1u << lane) - 1));
-        S.cand_key[slot] = key;
-      }
-    }
-  }
-  __syncthreads();   // every thread has read S.hist[prefix] before it is cleared
-  const int ncand = use_cand ? (int)S.cand_n : n;
-  kstamp(a.trace, 4);
-
-  // ---- digits 1 and 2 (10 bits each) over the candidates (or the segment)
-  int shift = 20;
-#pragma unroll 1
-  for (int d = 0; d < 2; ++d) {
-    const int nshift = 10 - 10 * d;                  // 10, then 0
-    for (int i = tid; i < 1024; i += kThreads) S.hist[i] = 0;
-    __syncthreads();
-    const int nr = (ncand + kThreads - 1) / kThreads;
-    for (int r = 0; r < nr; ++r) {
-      const int i = r * kThreads + tid;
-      bool v = i < ncand;
-      uint32_t key = 0;
-      if (v) key = use_cand ? S.cand_key[i] : key_at(i);
-      v = v && ((key >> shift) == prefix);
-      hist_add(S.hist, v, (key >> nshift) & 1023u);
-    }
-    kstamp(a.trace, 5 + 2 * d);
-    cluster_select(S, 1024, need, csize, rank, (d + 1) & 1);
-    prefix = (prefix << 10) | S.sel[(d + 1) & 1][0];
-    need = S.sel[(d + 1) & 1][1];
-    shift = nshift;
-    kstamp(a.trace, 6 + 2 * d);
-  }
-  const uint32_t T = prefix;     // the k-th largest key
-
-  // ---- counts of keys > T and == T per warp chunk (positions in order:
-  // warp w owns [w*chunk, (w+1)*chunk)), per CTA, shared with the cluster
-  const int chunk = ((n + kWarps - 1) / kWarps + 31) & ~31;
-  const int w_lo = min(warp * chunk, n), w_hi = min(w_lo + chunk, n);
-  uint32_t w_gt = 0, w_eq = 0;
-  for (int i = w_lo + lane; i < w_hi; i += 32) {
-    const uint32_t key = key_at(i);
-    w_gt += key > T;
-    w_eq += key == T;
-  }
+  // four keys starting at 4v (converted); entries at or past n are garbage
+  auto key4 = [&](int v) -> uint4 {
+    if (4 * v < ncache) return *reinterpret_cast<const uint4*>(&S.keys[4 * v]);
+    uint32_t q[4];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    w_gt += __shfl_xor_sync(0xffffffffu, w_gt, off);
-    w_eq += __shfl_xor_sync(0xffffffffu, w_eq, off);
+    for (int j = 0; j < 4; ++j) q[j] = 4 * v + j < n ? float_key(__ldcg(srow + 4 * v + j)) : 0u;
+    return make_uint4(q[0], q[1], q[2], q[3]);
+  };
+  auto nvalid = [&](int v) { return min(4, n - 4 * v); };
+
+  // ---- 1. keys in place, histogram of bits 31..20, cluster-wide bin B0
+#pragma unroll 2
+  for (int v = tid; v < nvec; v += kThreads) {
+    uint32_t q[4];
+    if (4 * v < ncache) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(&S.keys[4 * v]);
+      q[0] = float_key(__uint_as_float(raw.x));
+      q[1] = float_key(__uint_as_float(raw.y));
+      q[2] = float_key(__uint_as_float(raw.z));
+      q[3] = float_key(__uint_as_float(raw.w));
+      *reinterpret_cast<uint4*>(&S.keys[4 * v]) = make_uint4(q[0], q[1], q[2], q[3]);
+    } else {
+      const uint4 g = key4(v);
+      q[0] = g.x; q[1] = g.y; q[2] = g.z; q[3] = g.w;
+    }
+    const int nv = nvalid(v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (j < nv) atomicAdd(&S.hist[q[j] >> 20], 1u);
   }
-  if (lane == 0) {
-    S.warp_cnt[warp][0] = w_gt;
-    S.warp_cnt[warp][1] = w_eq;
+  kstamp(a.trace, csize, rank, 2);
+  cluster_select(S, kBins0, (uint32_t)k, csize, rank);
+  const uint32_t B0 = S.sel_bin, need0 = S.sel_need, c0 = S.sel_cnt;
+  kstamp(a.trace, csize, rank, 3);
+
+  // ---- 2. bitmap of the keys in bin B0 or above (segments held in smem):
+  // lanes 8i..8i+7 of a round hold the 32 keys of one word
+  const bool use_bits = n <= kCacheCap;               // uniform over the CTA
+  const int nwords = (n + 31) >> 5;                   // <= 512 = kThreads when use_bits
+  for (int i = tid; i < 2 * kBins; i += kThreads) (&S.lhist[0][0])[i] = 0;
+  if (tid == 0) S.gcount = 0;
+  if (use_bits) {
+    for (int base = warp * 32; base < nvec; base += kThreads) {
+      const int v = base + lane;
+      const bool inb = v < nvec;
+      const uint4 g = inb ? *reinterpret_cast<const uint4*>(&S.keys[4 * v]) : make_uint4(0, 0, 0, 0);
+      const uint32_t q[4] = {g.x, g.y, g.z, g.w};
+      const int nv = inb ? nvalid(v) : 0;
+      uint32_t m = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m |= (j < nv && (q[j] >> 20) >= B0) ? (1u << j) : 0u;
+      m <<= 4 * (lane & 7);
+      m |= __shfl_xor_sync(0xffffffffu, m, 1);
+      m |= __shfl_xor_sync(0xffffffffu, m, 2);
+      m |= __shfl_xor_sync(0xffffffffu, m, 4);
+      if ((lane & 7) == 0 && inb) S.bits[v >> 3] = m;
+    }
   }
   __syncthreads();
-  uint32_t gw = 0, ew = 0, tot_gt = 0, tot_eq = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const uint32_t g = S.warp_cnt[w][0], e = S.warp_cnt[w][1];
-    gw += w < warp ? g : 0u;
-    ew += w < warp ? e : 0u;
-    tot_gt += g;
-    tot_eq += e;
-  }
-  if (tid < (int)csize) {
-    if (csize == 1) {
-      S.counts[rank][0] = tot_gt;
-      S.counts[rank][1] = tot_eq;
-    } else {
-      st_dsmem_u32(mapa(&S.counts[rank][0], (uint32_t)tid), tot_gt);
-      st_dsmem_u32(mapa(&S.counts[rank][1], (uint32_t)tid), tot_eq);
+  const uint32_t myword = (use_bits && tid < nwords) ? S.bits[tid] : 0u;
+  const uint32_t* const mykeys = &S.keys[32 * tid];
+  kstamp(a.trace, csize, rank, 4);
+
+  // ---- 3. T, `need`, and this CTA's offsets in the cluster-wide order:
+  // out_base = keys the lower-ranked CTAs select, eq_base = their keys == T
+  uint32_t T, need, out_base = 0, eq_base = 0;
+  const bool gathered = c0 <= (uint32_t)kGatherCap;   // uniform over the cluster
+  if (gathered) {
+    // where this CTA's bin-B0 keys go in the gathered list: after those of
+    // lower ranks (their histograms still hold their counts of bin B0)
+    if (warp == 0) {
+      uint32_t hb = 0;
+      if (lane < (int)rank) hb = ld_dsmem_u32(mapa(&S.hist[B0], (uint32_t)lane));
+      hb = __reduce_add_sync(0xffffffffu, hb);
+      if (lane == 0) S.goff = hb;
     }
-  }
-  cluster_sync();
-  kstamp(a.trace, 9);
-  uint32_t out_base = 0, eq_base = 0;
-  for (uint32_t r = 0; r < rank; ++r) {
-    const uint32_t e = S.counts[r][1];
-    const uint32_t take = (eq_base >= need) ? 0u : min(e, need - eq_base);
-    out_base += S.counts[r][0] + take;
-    eq_base += e;
+    uint32_t ab = 0;                                  // keys of this segment above bin B0
+    for (int b = (int)B0 + 1 + tid; b < kBins0; b += kThreads) ab += S.hist[b];
+    ab = block_sum(ab, S.warp_tmp);                   // also publishes S.goff
+    const uint32_t goff = S.goff;
+    if (tid < (int)csize) {
+      if ((uint32_t)tid == rank) S.above[rank] = ab;
+      else st_dsmem_u32(mapa(&S.above[rank], (uint32_t)tid), ab);
+    }
+    auto send = [&](uint32_t key) {
+      const uint32_t slot = goff + atomicAdd(&S.gcount, 1u);
+      for (uint32_t r = 0; r < csize; ++r) {
+        if (r == rank) S.gather[slot] = key;
+        else st_dsmem_u32(mapa(&S.gather[slot], r), key);
+      }
+    };
+    if (use_bits) {
+      for (uint32_t w = myword; w; w &= w - 1) {
+        const uint32_t key = mykeys[__ffs(w) - 1];
+        if ((key >> 20) == B0) send(key);
+      }
+    } else {
+      for (int v = tid; v < nvec; v += kThreads) {
+        const uint4 g = key4(v);
+        const uint32_t q[4] = {g.x, g.y, g.z, g.w};
+        const int nv = nvalid(v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j < nv && (q[j] >> 20) == B0) send(q[j]);
+      }
+    }
+    // Last cluster barrier of this path: after it no CTA touches another's
+    // shared memory, so each may finish and exit on its own.
+    cluster_sync();
+    kstamp(a.trace, csize, rank, 5);
+    // the need0-th largest of the c0 gathered keys: two 10-bit digits, locally
+    for (int i = tid; i < (int)c0; i += kThreads)
+      atomicAdd(&S.lhist[0][(S.gather[i] >> 10) & 1023u], 1u);
+    __syncthreads();
+    if (warp == 0) warp_search_1024(S.lhist[0], need0, &S.sel_bin, &S.sel_need);
+    __syncthreads();
+    const uint32_t p1 = (B0 << 10) | S.sel_bin, n1 = S.sel_need;
+    for (int i = tid; i < (int)c0; i += kThreads) {
+      const uint32_t key = S.gather[i];
+      if ((key >> 10) == p1) atomicAdd(&S.lhist[1][key & 1023u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) warp_search_1024(S.lhist[1], n1, &S.sel_bin, &S.sel_need);
+    __syncthreads();
+    T = (p1 << 10) | S.sel_bin;
+    need = S.sel_need;
+    // gathered keys of lower ranks against T (> T in the high half, == T in
+    // the low half; both < 2^16)
+    uint32_t g = 0;
+    for (int i = tid; i < (int)goff; i += kThreads) {
+      const uint32_t key = S.gather[i];
+      g += (key > T ? 0x10000u : 0u) + (key == T ? 1u : 0u);
+    }
+    g = block_sum(g, S.warp_tmp);
+    uint32_t ab_before = 0;
+    for (uint32_t r = 0; r < rank; ++r) ab_before += S.above[r];
+    eq_base = g & 0xFFFFu;
+    out_base = ab_before + (g >> 16) + min(eq_base, need);
+    kstamp(a.trace, csize, rank, 6);
+  } else {
+    // the last two digits as cluster-wide histograms
+    uint32_t prefix = B0, nd = need0;
+    int shift = 20;
+#pragma unroll 1
+    for (int d = 0; d < 2; ++d) {
+      const int nshift = shift - 10;
+      for (int i = tid; i < kBins; i += kThreads) S.hist[i] = 0;
+      __syncthreads();
+      if (use_bits) {
+        for (uint32_t w = myword; w; w &= w - 1) {
+          const uint32_t key = mykeys[__ffs(w) - 1];
+          if ((key >> shift) == prefix) atomicAdd(&S.hist[(key >> nshift) & 1023u], 1u);
+        }
+      } else {
+#pragma unroll 2
+        for (int v = tid; v < nvec; v += kThreads) {
+          const uint4 g = key4(v);
+          const uint32_t q[4] = {g.x, g.y, g.z, g.w};
+          const int nv = nvalid(v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (j < nv && (q[j] >> shift) == prefix) atomicAdd(&S.hist[(q[j] >> nshift) & 1023u], 1u);
+        }
+      }
+      cluster_select(S, kBins, nd, csize, rank);
+      prefix = (prefix << 10) | S.sel_bin;
+      nd = S.sel_need;
+      shift = nshift;
+    }
+    T = prefix;
+    need = nd;
   }
 
-  // ---- ordered output: lane-interleaved rounds of 32 positions per warp;
-  // ballots give the order inside a round.  An equal key is taken while the
-  // number of equal keys before it (cluster-wide, in position order) < need.
-  uint32_t eq_rank = eq_base + ew;
-  const uint32_t eq_taken_before = (eq_base >= need) ? 0u : min(ew, need - eq_base);
-  uint32_t pos = out_base + gw + eq_taken_before;
-  const uint32_t lt_mask = (1u << lane) - 1;
-  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t key = i < w_hi ? key_at(i) : 0u;
-    const bool gt = i < w_hi && key > T;
-    const bool eq = i < w_hi && key == T;
-    const uint32_t em = __ballot_sync(0xffffffffu, eq);
-    const uint32_t my_eq_rank = eq_rank + __popc(em & lt_mask);
-    const bool sel = gt || (eq && my_eq_rank < need);
-    const uint32_t sm = __ballot_sync(0xffffffffu, sel);
-    if (sel) {
-      const uint32_t p = pos + __popc(sm & lt_mask);
-      if (p < (uint32_t)k) out[p] = lo + i;
+  // ---- 4. counts of keys > T and == T before each thread (bitmap) or warp
+  // (segment scan) in position order, and per CTA
+  const int cv = ((nvec + kWarps - 1) / kWarps + 31) & ~31;   // segment scan: vectors per warp
+  const int w_v0 = min(warp * cv, nvec), w_v1 = min(w_v0 + cv, nvec);
+  uint32_t gt_before, eq_before, tot_gt, tot_eq;
+  if (use_bits) {
+    uint32_t gt_t = 0, eq_t = 0;
+    for (uint32_t w = myword; w; w &= w - 1) {
+      const uint32_t key = mykeys[__ffs(w) - 1];
+      gt_t += key > T;
+      eq_t += key == T;
     }
-    pos += __popc(sm);
-    eq_rank += __popc(em);
+    uint32_t tot;   // > T in the high half, == T in the low half (both <= 16384)
+    const uint32_t before = block_excl_prefix((gt_t << 16) | eq_t, S.warp_tmp, &tot);
+    gt_before = before >> 16;
+    eq_before = before & 0xFFFFu;
+    tot_gt = tot >> 16;
+    tot_eq = tot & 0xFFFFu;
+  } else {
+    uint32_t w_gt = 0, w_eq = 0;
+#pragma unroll 2
+    for (int v = w_v0 + lane; v < w_v1; v += 32) {
+      const uint4 g = key4(v);
+      const uint32_t q[4] = {g.x, g.y, g.z, g.w};
+      const int nv = nvalid(v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        w_gt += (j < nv) & (q[j] > T);
+        w_eq += (j < nv) & (q[j] == T);
+      }
+    }
+    w_gt = __reduce_add_sync(0xffffffffu, w_gt);
+    w_eq = __reduce_add_sync(0xffffffffu, w_eq);
+    if (lane == 0) {
+      S.warp_cnt[warp][0] = w_gt;
+      S.warp_cnt[warp][1] = w_eq;
+    }
+    __syncthreads();
+    gt_before = eq_before = tot_gt = tot_eq = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const uint32_t gc = S.warp_cnt[w][0], ec = S.warp_cnt[w][1];
+      gt_before += w < warp ? gc : 0u;
+      eq_before += w < warp ? ec : 0u;
+      tot_gt += gc;
+      tot_eq += ec;
+    }
   }
-  kstamp(a.trace, 10);
-  cluster_sync();   // keep this CTA's smem alive until the cluster's remote accesses are done
-  kstamp(a.trace, 11);
+  if (!gathered) {
+    if (tid < (int)csize) {
+      if ((uint32_t)tid == rank) {
+        S.counts[rank][0] = tot_gt;
+        S.counts[rank][1] = tot_eq;
+      } else {
+        st_dsmem_u32(mapa(&S.counts[rank][0], (uint32_t)tid), tot_gt);
+        st_dsmem_u32(mapa(&S.counts[rank][1], (uint32_t)tid), tot_eq);
+      }
+    }
+    // Last cluster barrier of this path (see above).
+    cluster_sync();
+    for (uint32_t r = 0; r < rank; ++r) {
+      const uint32_t e = S.counts[r][1];
+      out_base += S.counts[r][0] + ((eq_base >= need) ? 0u : min(e, need - eq_base));
+      eq_base += e;
+    }
+  }
+  kstamp(a.trace, csize, rank, 7);
+
+  // ---- ordered output
+  uint32_t eq_rank = eq_base + eq_before;             // equal keys before this thread / warp
+  uint32_t pos = out_base + gt_before + ((eq_base >= need) ? 0u : min(eq_before, need - eq_base));
+  if (use_bits) {
+    for (uint32_t w = myword; w; w &= w - 1) {
+      const int b = __ffs(w) - 1;
+      const uint32_t key = mykeys[b];
+      const bool eq = key == T;
+      if (key > T || (eq && eq_rank < need)) {
+        if (pos < (uint32_t)k) out[pos] = lo + 32 * tid + b;
+        ++pos;
+      }
+      eq_rank += eq;
+    }
+  } else {
+    // lane L of a round holds positions 4(v0+L) .. +3: position order is
+    // lane-major, then j
+    const uint32_t lt = (1u << lane) - 1;
+    for (int v0 = w_v0; v0 < w_v1; v0 += 32) {
+      const int v = v0 + lane;
+      const bool inb = v < w_v1;
+      const uint4 g = inb ? key4(v) : make_uint4(0, 0, 0, 0);
+      const uint32_t q[4] = {g.x, g.y, g.z, g.w};
+      const int nv = inb ? nvalid(v) : 0;
+      bool gt[4], eq[4];
+      uint32_t e_before = 0, e_round = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        gt[j] = j < nv && q[j] > T;
+        eq[j] = j < nv && q[j] == T;
+        const uint32_t bl = __ballot_sync(0xffffffffu, eq[j]);
+        e_before += __popc(bl & lt);
+        e_round += __popc(bl);
+      }
+      bool sel[4];
+      uint32_t r_eq = eq_rank + e_before;
+      uint32_t s_before = 0, s_round = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sel[j] = gt[j] || (eq[j] && r_eq < need);
+        r_eq += eq[j];
+        const uint32_t bl = __ballot_sync(0xffffffffu, sel[j]);
+        s_before += __popc(bl & lt);
+        s_round += __popc(bl);
+      }
+      uint32_t p = pos + s_before;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (sel[j]) {
+          if (p < (uint32_t)k) out[p] = lo + 4 * v + j;
+          ++p;
+        }
+      }
+      pos += s_round;
+      eq_rank += e_round;
+    }
+  }
+  kstamp(a.trace, csize, rank, 8);
 }
 
 }  // namespace
