@@ -148,19 +148,27 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu capture, or None when the
-    kernel source changed since the counters were taken."""
+def kernel_traffic(kernel: str, workload: str, alg_bytes: int):
+    """DRAM bytes per launch of `kernel` on this launch's work, from a committed
+    ncu capture: the captured launch's DRAM bytes scaled by the ratio of
+    algorithmic bytes (the capture may be of a smaller batch of the same
+    workload, where traffic grows with the keys processed).  None when any
+    source of the kernel changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(f"{kernel}@{workload}")
     if not d:
         return None
-    src = os.path.join(ROOT, d["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["sha256"]:
+    h = hashlib.sha256()
+    for s in d["sources"]:
+        src = os.path.join(ROOT, s)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    if h.hexdigest() != d["sha256"]:
         return None
-    return d["dram_bytes_per_launch"]
+    return d["dram_bytes"] * alg_bytes / d["algorithmic_bytes"]
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -358,7 +366,7 @@ def run_ours(args):
              "mla": "mla_tc_kernel" if mla_tc else "mla_simt_kernel"}[dom]
     roof = {"kernel": kname, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak if peak else None, "peak_source": peak_kind,
-            "traffic": kernel_traffic(kname, args.workload),
+            "traffic": kernel_traffic(kname, args.workload, alg["bytes"]),
             "algorithmic_per_launch": alg["bytes"] if bound == "hbm" else alg["flops"]}
     stages = {}
     for k in avg:

@@ -10,9 +10,12 @@
 // splits the 576 dims between them: CTA r holds latent dims [256r, 256r+256)
 // and RoPE dims [32r, 32r+32) of Q (128 heads) and of every gathered key.
 //   * S_r = Q_r . KV_r^T (M=128 heads, N=64 keys, K=288) on the tensor cores.
-//   * The two partial logit tiles are exchanged through distributed shared
-//     memory; both CTAs form S = S_0 + S_1 (identical bits) and the same
-//     online softmax, so P is the same in both.
+//   * Each CTA sends its partial logit tile to the peer through distributed
+//     shared memory, as a per-row max plus 16-bit fixed-point distances to it
+//     (16.5 KB per 64 keys, one bulk copy).  Each CTA then forms
+//     z = S_own (exact fp32) + S_peer (decoded) and runs its own online
+//     softmax; the two sums differ only by the transport rounding, and each
+//     CTA's (max, sum) state normalises its own half of the value dims.
 //   * O_r += P . V_r with V_r = latent dims [256r, 256r+256) of the same
 //     gathered rows (M=128, N=256, K=64), P read from tensor memory.
 // No FLOP is done twice, every gathered byte is read once, and the 128 heads
