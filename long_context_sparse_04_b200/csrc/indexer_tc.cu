@@ -58,6 +58,7 @@ struct __align__(1024) IdxSmem {
   uint8_t q[2][NQ * kHI * kDI];
   float wq[kEpiWarps][kHI];                             // per epilogue warp: w' of its heads
   int32_t tile_row[kMaxCtaTiles][2];                    // physical row of each 64-key half, -1: none
+  int32_t tile_info[kMaxCtaTiles];                      // group << 2 | last tile of group << 1 | first
   int32_t tile_off[kMaxGroups + 1];
   int32_t scan_tmp[kThreads / 32];
   uint64_t full[num_stages<NQ>()], empty[num_stages<NQ>()];
@@ -223,6 +224,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         row = ok ? (int32_t)r : -1;
       }
       S.tile_row[i >> 1][i & 1] = row;
+      if ((i & 1) == 0) {
+        const int j = i >> 1;
+        S.tile_info[j] = (it.g << 2) | ((it.kt + 1 == it.ntiles || j + 1 == ntile) ? 2 : 0) |
+                         ((it.kt == 0 || j == 0) ? 1 : 0);
+      }
     }
   }
   __syncthreads();
@@ -231,79 +237,85 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   if (warp == 0) {
     // ------------------------------------------------------------ producer (lane 0): TMA only
     if (run && lane == 0) {
+      // A lean loop: one thread issues every load, so its instruction count
+      // per tile bounds the tile rate.
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_q);
-      TileIter it;
-      it.start(S.tile_off, a.n_groups, t_begin);
+      const bool tracing = a.trace != nullptr && blockIdx.x == 0;
+      int st = 0, qb = 0;
+      uint32_t ph = 1, qph = 1;                       // parity to wait for on empty / q_empty
       int qcount = 0, j = 0;
       bool alive = true;
-      for (; j < ntile && alive; ++j, it.next()) {
-        const int st = j % kStages;
-        if (j == 0 || it.kt == 0) {
-          const int qb = qcount & 1;
-          alive = mbar_wait(&S.q_empty[qb], ((qcount >> 1) & 1) ^ 1, a.status, 1);
-          if (!alive) break;
-          mbar_expect_tx(&S.q_full[qb], kQBytes);
-          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, it.g * NQ * kHI);
+      for (; j < ntile; ++j) {
+        const int info = S.tile_info[j];
+        const int2 rr = *reinterpret_cast<const int2*>(S.tile_row[j]);
+        if (info & 1) {
+          if (qcount > 0) { qb ^= 1; if (qb == 0) qph ^= 1; }
           ++qcount;
+          if (!(alive = mbar_wait(&S.q_empty[qb], qph, a.status, 1))) break;
+          mbar_expect_tx(&S.q_full[qb], kQBytes);
+          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, (info >> 2) * NQ * kHI);
         }
-        alive = mbar_wait(&S.empty[st], ((j / kStages) & 1) ^ 1, a.status, 2);
-        if (!alive) break;
-        istamp(a.trace, 0, j);
-        const int r0 = S.tile_row[j][0], r1 = S.tile_row[j][1];
-        const uint32_t bytes = (r0 >= 0 ? kKeyTileBytes / 2 : 0) + (r1 >= 0 ? kKeyTileBytes / 2 : 0);
+        if (!(alive = mbar_wait(&S.empty[st], ph, a.status, 2))) break;
+        if (tracing) istamp(a.trace, 0, j);
+        const uint32_t bytes = (rr.x >= 0 ? kKeyTileBytes / 2 : 0) + (rr.y >= 0 ? kKeyTileBytes / 2 : 0);
         if (bytes == 0) {
           mbar_arrive(&S.full[st]);
         } else {
           mbar_expect_tx(&S.full[st], bytes);
-          if (r0 >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, r0);
-          if (r1 >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, r1);
+          if (rr.x >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, rr.x);
+          if (rr.y >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, rr.y);
         }
-        istamp(a.trace, 1, j);
+        if (tracing) istamp(a.trace, 1, j);
+        if (++st == kStages) { st = 0; ph ^= 1; }
       }
       // tail: wait until the MMAs have released every stage and query buffer in
       // use, so no commit is still in flight to this CTA's shared memory at exit
       if (alive) {
-        for (int st = 0; st < kStages && st < j; ++st) {
-          const int last_use = (j - 1 - st) / kStages;
-          if (!mbar_wait(&S.empty[st], last_use & 1, a.status, 7)) break;
+        for (int s2 = 0; s2 < kStages && s2 < j; ++s2) {
+          const int last_use = (j - 1 - s2) / kStages;
+          if (!mbar_wait(&S.empty[s2], last_use & 1, a.status, 7)) break;
         }
-        for (int qb = 0; qb < 2 && qb < qcount; ++qb) {
-          const int last_use = (qcount - 1 - qb) >> 1;
-          if (!mbar_wait(&S.q_empty[qb], last_use & 1, a.status, 8)) break;
+        for (int q2 = 0; q2 < 2 && q2 < qcount; ++q2) {
+          const int last_use = (qcount - 1 - q2) >> 1;
+          if (!mbar_wait(&S.q_empty[q2], last_use & 1, a.status, 8)) break;
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && run) {
-      TileIter it;
-      it.start(S.tile_off, a.n_groups, t_begin);
+      // A lean loop (see the producer): descriptors are a base plus a stage or
+      // k-step offset in their start-address field (address >> 4).
       constexpr uint32_t idesc = idesc_f8_e4m3(N);
-      int qcount = -1;
+      const bool tracing = a.trace != nullptr && blockIdx.x == 0;
+      const uint64_t kd0 = sdesc_sw128(smem_u32(S.keys[0]), 16, 1024);
+      const uint64_t qd0 = sdesc_sw128(smem_u32(S.q[0]), 16, 1024);
+      constexpr uint64_t kStageStep = kKeyTileBytes >> 4, kQStep = kQBytes >> 4;
+      int st = 0, ab = 0, qb = 1;
+      uint32_t ph = 0, aph = 1, qph = 1;              // parity to wait for on full / acc_empty / q_full
       for (int j = 0; j < ntile; ++j) {
-        const bool first = (j == 0 || it.kt == 0);
-        if (first) {
-          ++qcount;
-          if (!mbar_wait(&S.q_full[qcount & 1], (qcount >> 1) & 1, a.status, 3)) break;
+        const int info = S.tile_info[j];
+        if (info & 1) {
+          qb ^= 1;
+          if (qb == 0) qph ^= 1;
+          if (!mbar_wait(&S.q_full[qb], qph, a.status, 3)) break;
         }
-        const int st = j % kStages, ab = j % kAcc;
-        if (!mbar_wait(&S.full[st], (j / kStages) & 1, a.status, 4)) break;
-        if (!mbar_wait(&S.acc_empty[ab], ((j / kAcc) & 1) ^ 1, a.status, 5)) break;
+        if (!mbar_wait(&S.full[st], ph, a.status, 4)) break;
+        if (tracing) istamp(a.trace, 5, j);
+        if (!mbar_wait(&S.acc_empty[ab], aph, a.status, 5)) break;
         tc_fence_after();
-        istamp(a.trace, 2, j);
-        const uint32_t ka = smem_u32(S.keys[st]);
-        const uint32_t qa = smem_u32(S.q[qcount & 1]);
+        if (tracing) istamp(a.trace, 2, j);
+        const uint64_t kd = kd0 + (uint64_t)st * kStageStep, qd = qd0 + (uint64_t)qb * kQStep;
+        const uint32_t d = tmem + ab * N;
 #pragma unroll
-        for (int k = 0; k < kDI / 32; ++k)
-          mma_f8(tmem + ab * N, sdesc_sw128(ka + 32 * k, 16, 1024), sdesc_sw128(qa + 32 * k, 16, 1024),
-                 idesc, k > 0);
+        for (int k = 0; k < kDI / 32; ++k) mma_f8(d, kd + 2 * k, qd + 2 * k, idesc, k > 0);
         mma_commit(&S.empty[st]);
         mma_commit(&S.acc_full[ab]);
-        istamp(a.trace, 3, j);
-        const bool last = (it.kt + 1 == it.ntiles) || (j + 1 == ntile);
-        if (last) mma_commit(&S.q_empty[qcount & 1]);
-        it.next();
+        if (info & 2) mma_commit(&S.q_empty[qb]);
+        if (tracing) istamp(a.trace, 3, j);
+        if (++st == kStages) { st = 0; ph ^= 1; }
+        if (++ab == kAcc) { ab = 0; aph ^= 1; }
       }
     }
   } else if (run) {
@@ -481,6 +493,25 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                       uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool indexer_tc_supported(const IndexerArgs& a) {
   if (a.idx_dtype != DSA_FP8_E4M3 || a.d_idx != kDI || a.n_idx_heads != kHI) return false;
