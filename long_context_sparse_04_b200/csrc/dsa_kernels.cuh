@@ -1,8 +1,6 @@
 // dsa_kernels.cuh - argument blocks and launchers of the DSA kernels.
 #pragma once
 
-#include <cuda.h>
-
 #include "dsa_common.cuh"
 
 namespace dsa {
@@ -76,12 +74,6 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream);
 bool mla_tc_supported(const MlaArgs& a);
 int mla_tc_splits(int num_rows);
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
-
-// Tensor maps (driver entry point looked up once).  A bf16 matrix [rows, cols],
-// row-major with no padding, box box_cols x box_rows, swizzle 0 / 64 / 128 bytes.
-bool tensor_maps_available();
-bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
-                       uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
 // Host-side error text of the calling thread.
 void set_error(const char* fmt, ...);
