@@ -110,6 +110,18 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels of one call are launched with programmatic stream serialization:
+// a kernel may start while its predecessor in the stream is still running.
+// pdl_wait() returns once every predecessor grid has completed and its memory
+// is visible; it must come before the first access to memory a predecessor
+// writes (or reads, for a later write).  Without the launch attribute it
+// returns at once.  pdl_launch_dependents() lets the next kernel start.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA (no multicast)
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar,
                                             int32_t x, int32_t y) {

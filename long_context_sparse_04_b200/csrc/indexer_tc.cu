@@ -148,6 +148,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   IdxSmem<NQ>& S = *reinterpret_cast<IdxSmem<NQ>*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  pdl_wait();
   trace_kernel(a.status, DSA_KERNEL_INDEXER_TC);
 
   // ---- schedule: exclusive scan of key tiles per group (every CTA, redundantly)

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
   const int unit = blockIdx.x >> 1;
   const int t = unit / a.splits, sp = unit % a.splits;
-  trace_kernel(a.status, DSA_KERNEL_MLA_TC);
+  pdl_launch_dependents();
 
   const int klen = a.row_klen[t];
   const int nsel = min(klen, a.topk);
@@ -152,17 +152,50 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // physical rows of the selected keys of this split (entries past nvalid are none)
-  const int32_t* idx = a.idx + (int64_t)t * a.topk + k0;
-  for (int i = threadIdx.x; i < nblk * kBlk; i += kThreads) {
-    int row = -1;
-    const int s = i < nvalid ? idx[i] : -1;
-    if (s >= 0 && s < klen) {
-      bool ok = true;
-      const int64_t r = a.map.row(seq, s, a.status, &ok);
-      row = ok ? (int32_t)r : -1;
+  // Q first: it does not depend on the selection (the gather warps arrive on
+  // q_full for these pieces once the barrier init is visible, below)
+  if (warp < 4 && nblk > 0) {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
+    for (int i = 0; i < kPieces; ++i) {
+      const int qi = i * 128 + threadIdx.x;
+      const int h = qi / kPieces, c = qi - h * kPieces;
+      if (c < 32) {
+        cp_async_16(S.q[c >> 3] + sw128_off(h, c & 7), qrow + h * kD + 256 * rank + 8 * c);
+      } else {
+        cp_async_16(S.q_rope + sw64_off(h, c - 32), qrow + h * kD + kDC + 32 * rank + 8 * (c - 32));
+      }
     }
-    S.rows[i] = row;
+  }
+  // The selection comes from the previous kernel: everything above (barriers,
+  // TMEM, the Q load) overlaps its tail.
+  pdl_wait();
+  trace_kernel(a.status, DSA_KERNEL_MLA_TC);
+  // physical rows of the selected keys of this split (entries past nvalid are
+  // none): all index loads of a thread first, then all its block-table loads
+  {
+    constexpr int kPer = (kMaxKeys + kThreads - 1) / kThreads;
+    const int32_t* idx = a.idx + (int64_t)t * a.topk + k0;
+    const int nk = nblk * kBlk;
+    int sv[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      sv[u] = i < nvalid ? __ldg(idx + i) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      if (i < nk) {
+        int row = -1;
+        const int sk = sv[u];
+        if (sk >= 0 && sk < klen) {
+          bool ok = true;
+          const int64_t r = a.map.row(seq, sk, a.status, &ok);
+          row = ok ? (int32_t)r : -1;
+        }
+        S.rows[i] = row;
+      }
+    }
   }
   __syncthreads();
   for (int b = threadIdx.x; b < nblk; b += kThreads) {
@@ -180,16 +213,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     // ------------------------------------------------------------ gather (128 threads)
     const int tid = threadIdx.x;
     if (nblk > 0) {
-      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
-      for (int i = 0; i < kPieces; ++i) {
-        const int qi = i * 128 + tid;
-        const int h = qi / kPieces, c = qi - h * kPieces;
-        if (c < 32) {
-          cp_async_16(S.q[c >> 3] + sw128_off(h, c & 7), qrow + h * kD + 256 * rank + 8 * c);
-        } else {
-          cp_async_16(S.q_rope + sw64_off(h, c - 32), qrow + h * kD + kDC + 32 * rank + 8 * (c - 32));
-        }
-      }
       cp_async_mbar_arrive(&S.q_full);        // arrives when this thread's Q pieces land
       const __nv_bfloat16* lat = static_cast<const __nv_bfloat16*>(a.latent);
       bool alive = true;
@@ -464,6 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
 __global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
   // thread i: value dims 4i..4i+3, produced by CTA rank (4i >= 256) with that
   // CTA's own softmax state (m, l) of each split
+  pdl_wait();                                // the partials come from the attention kernel
   trace_kernel(a.status, DSA_KERNEL_MLA_COMBINE);
   const int th = blockIdx.x;
   const int t = th / kH, h = th % kH;
@@ -540,21 +564,31 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr2[1];
+  cudaLaunchAttribute attr2[2];
   attr2[0].id = cudaLaunchAttributeClusterDimension;
   attr2[0].val.clusterDim.x = 2;
   attr2[0].val.clusterDim.y = 1;
   attr2[0].val.clusterDim.z = 1;
+  attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr2[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr2;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, a, keys_per_split);
   if (e != cudaSuccess) {
     set_error("mla_tc launch: %s", cudaGetErrorString(e));
     return DSA_ERR_CUDA;
   }
   if (a.splits > 1) {
-    mla_combine_kernel<<<a.num_rows * kH, 128, 0, stream>>>(a);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cc = {};
+    cc.gridDim = dim3((unsigned)(a.num_rows * kH));
+    cc.blockDim = dim3(128);
+    cc.stream = stream;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cc.attrs = pdl;
+    cc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cc, mla_combine_kernel, a);
     if (e != cudaSuccess) {
       set_error("mla_combine launch: %s", cudaGetErrorString(e));
       return DSA_ERR_CUDA;

@@ -34,6 +34,7 @@ __device__ __forceinline__ void store_elem(__nv_bfloat16* p, int64_t i, float v)
 template <typename KT>
 __global__ void __launch_bounds__(128) indexer_simt_kernel(IndexerArgs a) {
   extern __shared__ float sm[];
+  pdl_wait();
   trace_kernel(a.status, DSA_KERNEL_INDEXER_SIMT);
   const int t = blockIdx.y;
   const int H = a.n_idx_heads, D = a.d_idx;
@@ -68,6 +69,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) mla_simt_kernel(MlaArgs a) {
   constexpr int HB = 8, KC = 16;
   extern __shared__ float sm[];
+  pdl_wait();
   trace_kernel(a.status, DSA_KERNEL_MLA_SIMT);
   const int t = blockIdx.x;
   const int h0 = blockIdx.y * HB;

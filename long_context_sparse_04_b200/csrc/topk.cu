@@ -213,6 +213,8 @@ __device__ void cluster_select(TopkSmem& S, int nbins, uint32_t need, uint32_t c
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smraw);
+  pdl_launch_dependents();
+  pdl_wait();                                // the scores come from the previous kernel
   trace_kernel(a.status, DSA_KERNEL_TOPK);
   const uint32_t csize = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
@@ -570,13 +572,15 @@ dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, topk_kernel, a);
   if (e != cudaSuccess) {
     set_error("topk launch: %s", cudaGetErrorString(e));
