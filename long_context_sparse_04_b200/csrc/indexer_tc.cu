@@ -63,7 +63,7 @@ struct __align__(1024) IdxSmem {
   int32_t scan_tmp[kThreads / 32];
   uint64_t full[num_stages<NQ>()], empty[num_stages<NQ>()];
   uint64_t q_full[2], q_empty[2];
-  uint64_t acc_full[4], acc_empty[4];
+  uint64_t acc_empty[4];
   uint32_t tmem_base;
 };
 
@@ -191,7 +191,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       mbar_init(&S.q_empty[i], 1);
     }
     for (int i = 0; i < 4; ++i) {
-      mbar_init(&S.acc_full[i], 1);
       mbar_init(&S.acc_empty[i], 4 * NQ);     // the warps of one epilogue set
     }
     fence_mbar_init();
@@ -312,8 +311,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const uint32_t d = tmem + ab * N;
 #pragma unroll
         for (int k = 0; k < kDI / 32; ++k) mma_f8(d, kd + 2 * k, qd + 2 * k, idesc, k > 0);
-        mma_commit(&S.empty[st]);
-        mma_commit(&S.acc_full[ab]);
+        mma_commit(&S.empty[st]);           // stage free, and accumulator ab ready
         if (info & 2) mma_commit(&S.q_empty[qb]);
         if (tracing) istamp(a.trace, 3, j);
         if (++st == kStages) { st = 0; ph ^= 1; }
@@ -359,7 +357,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         if (rr >= 0 && pr < a.map.num_tokens) ks = __ldg(a.k_scale + pr);
       }
       const int ab = j % kAcc;
-      dead = dead || !mbar_wait(&S.acc_full[ab], (j / kAcc) & 1, a.status, 6);
+      // the stage's barrier completes when the tile's MMAs are done
+      dead = dead || !mbar_wait(&S.empty[j % kStages], (j / kStages) & 1, a.status, 6);
       tc_fence_after();
       if (threadIdx.x == 64) istamp(a.trace, 4, j);
       const uint32_t col = tmem + lane_off + ab * N + qi * kHI;
