@@ -223,14 +223,21 @@ def row_layout(cfg: DSAConfig):
 # whole workload
 # ----------------------------------------------------------------------------
 
-def generate(cfg: DSAConfig, with_q: bool = True, threads: int = 8) -> dict:
+def generate(cfg: DSAConfig, with_q: bool = True, threads: int = 8, rows=None) -> dict:
     """All inputs of one workload as host numpy arrays (storage formats).
 
     Keys: row_seq, row_klen, q_idx, q_scale, w, k_idx, k_scale, latent, q,
     cache (seq_start | block_table, page_size, num_pages), topk, d_c, d_r,
     sm_scale, idx_dtype, mla_dtype, n_heads, h_idx, d_idx, cfg.
+
+    rows: a subset of the workload's query rows (their indices), or None for
+    all.  Every query row is seeded on its own, so a subset's rows are
+    bit-identical to the same rows of the whole workload; the caches are always
+    generated whole.
     """
     row_seq, row_klen = row_layout(cfg)
+    qrows = np.arange(row_seq.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
+    row_seq, row_klen = row_seq[qrows], row_klen[qrows]
     T = row_seq.shape[0]
     ctx = context_lengths(cfg)
     nblk = [(int(c) + BLOCK - 1) // BLOCK for c in ctx]
@@ -287,19 +294,19 @@ def generate(cfg: DSAConfig, with_q: bool = True, threads: int = 8) -> dict:
     with ThreadPoolExecutor(max_workers=threads) as ex:
         list(ex.map(fill, jobs))
 
-    qf = qidx_rows_f32(cfg, range(T))
+    qf = qidx_rows_f32(cfg, qrows)
     if cfg.fp8:
         q_idx, q_scale = to_e4m3_rows(qf)
     else:
         q_idx, q_scale = qf, None
-    w = w_rows(cfg, range(T))
+    w = w_rows(cfg, qrows)
     inp = dict(row_seq=row_seq, row_klen=row_klen, q_idx=q_idx, q_scale=q_scale, w=w,
                k_idx=k_idx, k_scale=k_scale, latent=latent, cache=cache,
                topk=cfg.topk, d_c=cfg.d_c, d_r=cfg.d_r, sm_scale=cfg.sm_scale,
                idx_dtype="e4m3" if cfg.fp8 else "f32", mla_dtype="bf16" if cfg.bf16 else "f32",
                n_heads=cfg.n_heads, h_idx=cfg.h_idx, d_idx=cfg.d_idx, cfg=cfg)
     if with_q:
-        chunks = [range(i, min(T, i + 256)) for i in range(0, T, 256)]
+        chunks = [qrows[i: i + 256] for i in range(0, T, 256)]
         with ThreadPoolExecutor(max_workers=threads) as ex:
             parts = list(ex.map(lambda r: q_rows(cfg, r), chunks))
         inp["q"] = np.concatenate(parts) if parts else None
