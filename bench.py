@@ -6,7 +6,11 @@
 A step is one pass of all three stages (indexer -> top-k -> sparse MLA) over
 one batch of the workload: for the default 128K paged decode workload, 16
 sequences x 2 query rows with contexts drawn from [98304, 131072], one
-dsa_decode_step call.  The metric is query-tokens/s of one DSA layer.
+dsa_decode_step call; for the prefill workloads (--workload prefill_8k or
+prefill_64k), one dsa_forward call over the whole causal sequence.  The metric
+is query-tokens/s of one DSA layer.  The per-stage breakdown comes from an
+untimed pass: events the library records between its launches (decode), or
+the three stage calls over the whole batch (prefill).
 
 Under torchrun each rank runs its own batch (different seed, same shapes):
 weak scaling, no collective on the data path; the barrier and the max over
@@ -276,6 +280,17 @@ def run_ours(args):
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     out = torch.empty((T, wl.H, wl.d_c), dtype=wl.out_dtype(), device=dev)
     lse = torch.empty((T, wl.H), dtype=torch.float32, device=dev)
+    prefill = bool(cfg.prefill)
+    op = N.DSA_OP_FORWARD if prefill else N.DSA_OP_DECODE_STEP
+    idx_out = torch.empty((T, wl.topk), dtype=torch.int32, device=dev) if prefill else None
+
+    def step():
+        # one pass of the whole hot path over the batch: the fused decode call,
+        # or the chunked prefill forward
+        if prefill:
+            wl.forward(out=out, lse=lse, idx=idx_out)
+        else:
+            wl.decode_step(out=out, lse=lse)
 
     def barrier():
         if world > 1:
@@ -283,10 +298,10 @@ def run_ours(args):
 
     for _ in range(max(args.warmup, 0)):
         flush.zero_()
-        wl.decode_step(out=out, lse=lse)
+        step()
     torch.cuda.synchronize(dev)
-    st = wl.status(N.DSA_OP_DECODE_STEP)
-    ran = wl.kernels_ran(N.DSA_OP_DECODE_STEP)
+    st = wl.status(op)
+    ran = wl.kernels_ran(op)
     assert st == (0, -1), f"device status {st}"
 
     clocks = ClockSampler(dev.index if dev.index is not None else 0)
@@ -295,9 +310,9 @@ def run_ours(args):
     # samples (10 Hz) are taken under this load; the timed steps follow at once
     t_end = time.perf_counter() + 1.5
     while time.perf_counter() < t_end:
-        for _ in range(20):
+        for _ in range(20 if not prefill else 1):
             flush.zero_()
-            wl.decode_step(out=out, lse=lse)
+            step()
         torch.cuda.synchronize(dev)
     barrier()
     torch.cuda.synchronize(dev)
@@ -307,29 +322,51 @@ def run_ours(args):
     for _ in range(args.steps):
         flush.zero_()
         step_ev[0].record(stream)
-        wl.decode_step(out=out, lse=lse)
+        step()
         step_ev[1].record(stream)
         torch.cuda.synchronize(dev)
         step_ms.append(step_ev[0].elapsed_time(step_ev[1]))
     barrier()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
-    # per-stage breakdown (untimed for the headline): the library records
-    # events between its launches
-    N.dsa_set_stage_events([e.cuda_event for e in ev])
+    # per-stage breakdown (untimed for the headline)
     stage_ms = {"indexer": [], "topk": [], "mla": []}
-    for _ in range(args.steps):
-        flush.zero_()
-        wl.decode_step(out=out, lse=lse)
-        torch.cuda.synchronize(dev)
-        stage_ms["indexer"].append(ev[0].elapsed_time(ev[1]))
-        stage_ms["topk"].append(ev[1].elapsed_time(ev[2]))
-        stage_ms["mla"].append(ev[2].elapsed_time(ev[3]))
-    N.dsa_set_stage_events([])
+    if prefill:
+        # the three stage calls over the whole batch (the forward runs them
+        # per 512-row chunk)
+        scores = torch.empty((T, wl.ld), dtype=torch.float32, device=dev)
+        for _ in range(args.steps):
+            flush.zero_()
+            ev[0].record(stream)
+            wl.indexer(scores)
+            ev[1].record(stream)
+            wl.topk_(scores, idx_out)
+            ev[2].record(stream)
+            wl.mla(idx_out, out, lse)
+            ev[3].record(stream)
+            torch.cuda.synchronize(dev)
+            stage_ms["indexer"].append(ev[0].elapsed_time(ev[1]))
+            stage_ms["topk"].append(ev[1].elapsed_time(ev[2]))
+            stage_ms["mla"].append(ev[2].elapsed_time(ev[3]))
+        del scores
+    else:
+        # the library records events between its launches
+        N.dsa_set_stage_events([e.cuda_event for e in ev])
+        for _ in range(args.steps):
+            flush.zero_()
+            wl.decode_step(out=out, lse=lse)
+            torch.cuda.synchronize(dev)
+            stage_ms["indexer"].append(ev[0].elapsed_time(ev[1]))
+            stage_ms["topk"].append(ev[1].elapsed_time(ev[2]))
+            stage_ms["mla"].append(ev[2].elapsed_time(ev[3]))
+        N.dsa_set_stage_events([])
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     value = throughput(world, T, args.steps, total_ms)
-    launches_per_step = 3 + (1 if ran & N.DSA_KERNEL_MLA_COMBINE else 0)
+    if prefill:   # three kernels per 512-row chunk, no split combine
+        launches_per_step = 3 * ((T + 511) // 512)
+    else:
+        launches_per_step = 3 + (1 if ran & N.DSA_KERNEL_MLA_COMBINE else 0)
 
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
@@ -346,7 +383,7 @@ def run_ours(args):
             e0.record(stream)
             for k, v in host_in.items():
                 getattr(wl, k).copy_(v, non_blocking=True)
-            wl.decode_step(out=out, lse=lse)
+            step()
             host_out.copy_(out, non_blocking=True)
             host_lse.copy_(lse, non_blocking=True)
             e1.record(stream)
@@ -368,6 +405,14 @@ def run_ours(args):
         achieved = alg["flops"] / (avg[dom] / 1e3) / 1e12
         peak = peaks.get("bf16_tflops")
         unit = "TFLOP/s"
+    elif dom == "indexer" and prefill:
+        # FP8 contraction: no measured fp8 peak; the nominal fp8/bf16 ratio (2)
+        # times the measured bf16 peak
+        bound = "tensor"
+        achieved = alg["flops"] / (avg[dom] / 1e3) / 1e12
+        peak = 2.0 * peaks.get("bf16_tflops") if peaks.get("bf16_tflops") else None
+        unit = "TFLOP/s"
+        peak_kind = peak_kind + " (bf16 x 2, the nominal fp8/bf16 ratio)"
     else:
         bound = "hbm"
         achieved = alg["bytes"] / (avg[dom] / 1e3) / 1e9
