@@ -371,7 +371,8 @@ def run_ours(args):
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("q_idx", "q_scale", "w", "q", "row_klen")}
+        host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("q_idx", "q_scale", "w", "q", "row_klen")
+                   if getattr(wl, k) is not None}
         host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host_in.values())
@@ -400,7 +401,17 @@ def run_ours(args):
     dom = max(avg, key=avg.get)
     alg = algorithmic(cfg_r, inp, dom)
     mla_tc = bool(ran & N.DSA_KERNEL_MLA_TC)
-    if dom == "mla":
+    idx_tc = bool(ran & N.DSA_KERNEL_INDEXER_TC)
+    simt = (dom == "mla" and not mla_tc) or (dom == "indexer" and not idx_tc)
+    if simt:
+        # CUDA-core fp32 kernels: 148 SMs x 128 fp32 lanes x 2 FLOP (FMA) at
+        # the maximum SM clock
+        bound = "alu"
+        achieved = alg["flops"] / (avg[dom] / 1e3) / 1e12
+        peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        unit = "TFLOP/s"
+        peak_kind = "derived (SM count x fp32 lanes x 2 x max SM clock)"
+    elif dom == "mla":
         bound = "tensor"
         achieved = alg["flops"] / (avg[dom] / 1e3) / 1e12
         peak = peaks.get("bf16_tflops")
@@ -418,7 +429,7 @@ def run_ours(args):
         achieved = alg["bytes"] / (avg[dom] / 1e3) / 1e9
         peak = peaks.get("hbm_gbs")
         unit = "GB/s"
-    kname = {"indexer": "indexer_tc_kernel", "topk": "topk_kernel",
+    kname = {"indexer": "indexer_tc_kernel" if idx_tc else "indexer_simt_kernel", "topk": "topk_kernel",
              "mla": "mla_tc_kernel" if mla_tc else "mla_simt_kernel"}[dom]
     roof = {"kernel": kname, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak if peak else None, "peak_source": peak_kind,
