@@ -141,8 +141,9 @@ const char* dsa_last_error(void);
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t dsa_version(void);
 
-/* Bytes of workspace `op` needs for these dimensions and rows (host only; no
- * CUDA call).  Returns 0 for invalid arguments. */
+/* Bytes of workspace `op` needs for these dimensions and rows (host only; it
+ * reads the current device's SM count, which sets the decode key splits, and
+ * uses 148 when no device is present).  Returns 0 for invalid arguments. */
 size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op);
 
 /* Zero the device status word at the head of `ws` (async on stream). */

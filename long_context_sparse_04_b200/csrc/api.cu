@@ -22,6 +22,37 @@ static void stage_event(int i, cudaStream_t s) {
 
 long long* trace_buffer() { return g_trace; }
 
+dsa_status set_smem_limit_once(const void* fn, size_t bytes, std::atomic<bool> (&done)[kMaxDevices]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_error("no current CUDA device");
+    return DSA_ERR_CUDA;
+  }
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && done[dev].load(std::memory_order_acquire)) return DSA_OK;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) {
+    set_error("cannot allow %zu bytes of shared memory: %s", bytes, cudaGetErrorString(e));
+    return DSA_ERR_CUDA;
+  }
+  if (cached) done[dev].store(true, std::memory_order_release);
+  return DSA_OK;
+}
+
+int device_sm_count() {
+  static std::atomic<int> cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 void set_error(const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);

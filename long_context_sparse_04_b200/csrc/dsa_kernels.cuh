@@ -1,6 +1,8 @@
 // dsa_kernels.cuh - argument blocks and launchers of the DSA kernels.
 #pragma once
 
+#include <atomic>
+
 #include "dsa_common.cuh"
 
 namespace dsa {
@@ -74,6 +76,16 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream);
 bool mla_tc_supported(const MlaArgs& a);
 int mla_tc_splits(int num_rows);
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
+
+// Per-device host state.  Kernel attributes and device properties belong to a
+// device, so a process that drives several GPUs sets and caches them per
+// device (the current one at the call).
+constexpr int kMaxDevices = 128;
+// Raises the dynamic shared-memory limit of kernel `fn` to `bytes` on the
+// current device, once per device (`done` is the kernel's flag array).
+dsa_status set_smem_limit_once(const void* fn, size_t bytes, std::atomic<bool> (&done)[kMaxDevices]);
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
 
 // Host-side error text of the calling thread.
 void set_error(const char* fmt, ...);

@@ -428,29 +428,12 @@ bool make_tmap_rows128(CUtensorMap* m, const void* base, uint64_t rows, uint32_t
   return r == CUDA_SUCCESS;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int NQ>
 dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(IdxSmem<NQ>) + 1024;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(indexer_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess) {
-      set_error("indexer_tc: cannot set %zu bytes of shared memory", smem);
-      return DSA_ERR_CUDA;
-    }
-    attr = true;
-  }
+  static std::atomic<bool> attr[kMaxDevices] = {};
+  if (dsa_status st = set_smem_limit_once(reinterpret_cast<const void*>(indexer_tc_kernel<NQ>), smem, attr))
+    return st;
   CUtensorMap tm_k;
   if (!make_tmap_rows128(&tm_k, a.idx_k, (uint64_t)a.map.num_tokens, 64)) {
     set_error("indexer_tc: cuTensorMapEncodeTiled failed");
@@ -482,7 +465,7 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     // tiles are at most groups x ceil(max_klen / 128); a CTA takes at most kMaxCtaTiles
     const int64_t tiles = (int64_t)ng * ((a.max_klen + kTileKeys - 1) / kTileKeys);
     const int64_t need = (tiles + kMaxCtaTiles - 1) / kMaxCtaTiles;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, std::max<int64_t>(num_sms(), need)));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, std::max<int64_t>(device_sm_count(), need)));
     indexer_tc_kernel<NQ><<<grid, kThreads, smem, stream>>>(tm_k, tq, t);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {

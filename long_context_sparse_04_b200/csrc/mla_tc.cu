@@ -514,17 +514,6 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
   if (threadIdx.x == 0 && a.lse) a.lse[(int64_t)t * kH + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 }  // namespace
 
 bool mla_tc_supported(const MlaArgs& a) {
@@ -535,7 +524,7 @@ bool mla_tc_supported(const MlaArgs& a) {
 // Key splits of a decode batch: enough (row, split) CTA pairs to cover the SMs once.
 int mla_tc_splits(int num_rows) {
   if (num_rows <= 0) return 1;
-  const int pairs = sm_count() / 2;
+  const int pairs = device_sm_count() / 2;
   int s = 1;
   while (s < 8 && (int64_t)num_rows * s * 2 <= pairs) s <<= 1;
   return s;
@@ -549,15 +538,9 @@ size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits) {
 dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
   const size_t smem = sizeof(MlaSmem) + 1024;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess) {
-      set_error("mla_tc: cannot set %zu bytes of shared memory", smem);
-      return DSA_ERR_CUDA;
-    }
-    attr = true;
-  }
+  static std::atomic<bool> attr[kMaxDevices] = {};
+  if (dsa_status st = set_smem_limit_once(reinterpret_cast<const void*>(mla_tc_kernel), smem, attr))
+    return st;
   const int keys_per_split = (int)(ceil_div64(ceil_div64(a.topk, a.splits), kBlk) * kBlk);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.num_rows * a.splits * 2));

@@ -560,13 +560,9 @@ dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   int csize = 1;
   while (csize < kMaxCluster && (int64_t)csize * kCacheCap < (int64_t)max_klen) csize <<= 1;
   const size_t smem = sizeof(TopkSmem);
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_done = true;
-  }
+  static std::atomic<bool> attr_done[kMaxDevices] = {};
+  if (dsa_status st = set_smem_limit_once(reinterpret_cast<const void*>(topk_kernel), smem, attr_done))
+    return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.num_rows * csize));
   cfg.blockDim = dim3(kThreads);
