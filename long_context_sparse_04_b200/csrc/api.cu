@@ -1,6 +1,6 @@
 // api.cu - the C ABI of the DSA forward path: argument checks, workspace
 // planning, kernel selection and launches.  No entry point allocates device
-// memory or synchronises (except dsa_read_device_status).
+// memory; only dsa_read_device_status and dsa_read_kernel_trace synchronise.
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>

@@ -17,11 +17,15 @@
 // shared memory, so the loops below never wait on a dependent global load.
 // Roles (576 threads):
 //   warp 0      producer (one thread): TMA of the two 64-row key boxes (a box
-//               never crosses a 64-token page) into a 6-stage ring, and of the
-//               group's queries (N x 128 B) into a double buffer.
+//               never crosses a 64-token page) into a 10-stage ring (6 when
+//               N = 256), and of the group's queries (N x 128 B) into a double
+//               buffer.  Per-tile flags computed in the prologue (first / last
+//               tile of its group) keep this loop short.
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
-//               into one of four (N <= 128) or two TMEM accumulators.
+//               into one of four (N <= 128) or two TMEM accumulators; one
+//               commit per tile frees the key stage and tells the epilogue
+//               that the accumulator is ready.
 //   warps 2-17  epilogue in 16/(4*NQ) sets that take alternate tiles (one
 //               set's TMEM-load latency overlaps another's math): tcgen05.ld
 //               of the accumulator (lane = key), ReLU, head-weighted sum with w'
