@@ -180,23 +180,63 @@ def _plant_targets(cfg: DSAConfig, seq: int, chunk: int):
     return out
 
 
+def key_chunk_f32(cfg: DSAConfig, seq: int, chunk: int):
+    """Keys [1024*chunk, 1024*chunk + 1024) of sequence `seq` before the storage
+    casts: (k_I float32 [1024, d_I], latent float32 [1024, d_c+d_r])."""
+    k = _normal(cfg.seed, TID_KIDX, (seq, chunk), (CHUNK, cfg.d_idx), cfg.std_kidx)
+    for off, tgt, head in _plant_targets(cfg, seq, chunk):
+        qv = qidx_rows_f32(cfg, [tgt])[0, head]
+        k[off] = np.float32(4.0 * math.sqrt(cfg.d_idx)) * qv / np.float32(np.linalg.norm(qv))
+    lat = _normal(cfg.seed, TID_LATENT, (seq, chunk), (CHUNK, cfg.d_qk), cfg.std_kv)
+    return k, lat
+
+
 def key_chunk(cfg: DSAConfig, seq: int, chunk: int):
     """Keys [1024*chunk, 1024*chunk + 1024) of sequence `seq`, both caches.
 
     Returns (k_idx codes or f32 [1024, d_I], k_scale [1024] or None,
     latent [1024, d_c+d_r] in storage format).
     """
-    k = _normal(cfg.seed, TID_KIDX, (seq, chunk), (CHUNK, cfg.d_idx), cfg.std_kidx)
-    for off, tgt, head in _plant_targets(cfg, seq, chunk):
-        qv = qidx_rows_f32(cfg, [tgt])[0, head]
-        k[off] = np.float32(4.0 * math.sqrt(cfg.d_idx)) * qv / np.float32(np.linalg.norm(qv))
-    lat = _normal(cfg.seed, TID_LATENT, (seq, chunk), (CHUNK, cfg.d_qk), cfg.std_kv)
+    k, lat = key_chunk_f32(cfg, seq, chunk)
     if cfg.fp8:
         kc, ks = to_e4m3_rows(k)
     else:
         kc, ks = k, None
     lat = to_bf16_bits(lat) if cfg.bf16 else lat
     return kc, ks, lat
+
+
+def token_keys(cfg: DSAConfig, tok_seq, tok_pos):
+    """The generator's keys of tokens (tok_seq[n], tok_pos[n]) before the FP8
+    cast: (k_I float32 [n, d_I], latent [n, d_c+d_r] in storage format).  These
+    are what a cache append of those tokens takes as input."""
+    tok_seq = np.asarray(tok_seq, dtype=np.int64)
+    tok_pos = np.asarray(tok_pos, dtype=np.int64)
+    n = tok_seq.shape[0]
+    k = np.zeros((n, cfg.d_idx), np.float32)
+    lat = np.zeros((n, cfg.d_qk), np.float32)
+    cache = {}
+    for i in range(n):
+        key = (int(tok_seq[i]), int(tok_pos[i]) // CHUNK)
+        if key not in cache:
+            cache = {key: key_chunk_f32(cfg, *key)}
+        kc, lc = cache[key]
+        k[i] = kc[tok_pos[i] % CHUNK]
+        lat[i] = lc[tok_pos[i] % CHUNK]
+    return k, (to_bf16_bits(lat) if cfg.bf16 else lat)
+
+
+def new_tokens(cfg: DSAConfig):
+    """The tokens a decode step of the workload appends before it attends: the
+    last rows_per_seq positions of every sequence (prefill: every position).
+    Returns (tok_seq int32 [n], tok_pos int32 [n])."""
+    ctx = context_lengths(cfg)
+    if cfg.prefill:
+        return np.zeros(cfg.seq_len, np.int32), np.arange(cfg.seq_len, dtype=np.int32)
+    nq = cfg.rows_per_seq
+    seq = np.repeat(np.arange(cfg.n_seqs, dtype=np.int32), nq)
+    j = np.tile(np.arange(nq), cfg.n_seqs)
+    return seq, (ctx[seq] - nq + j).astype(np.int32)
 
 
 def context_lengths(cfg: DSAConfig) -> np.ndarray:

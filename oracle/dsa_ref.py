@@ -28,6 +28,16 @@ section and equation on that page):
   here in absorbed form: the query already carries W_UK, so a logit is
   sm_scale * (q[t,i] . [c_s || k^R_s]) over the 576 (or d_c + d_R) latent
   dims and the output is the latent sum_s p_s c_s (width d_c).
+* same page, item "Native FP8 Precision", with "Sparse Attention in Large
+  Language Models: Architecture Evolution and Engineering Practice", section 4,
+  item "Memory Management and KV Cache Optimization" (paged caches), and
+  "Sparse Attention Architectures for Long-Context Inference: Evolution and
+  Engineering Practices", section 6, item "Incremental inference adaptation"
+  (each decoding step writes its new tokens into the caches): the cache
+  append.  New indexer keys are quantised to e4m3 with one fp32 scale per
+  token (an encoder written from the OCP definition: nearest value, ties to
+  the even code, saturating at +-448) and written with their latent rows at
+  the rows the block table gives.
 * section "The Classical Multi-Head Latent Attention (MLA) Mechanism", logit
   equation A_{t,s,i}: the dense MLA that sparse MLA must equal when k covers
   every visible key, and the un-absorbed form used for the absorbed ==
@@ -267,3 +277,123 @@ def dsa_forward_rows(inp: dict, rows, topk: int | None = None):
         res["out"].append(o)
         res["lse"].append(lse)
     return res
+
+
+# ----------------------------------------------------------------------------
+# Cache append: FP8 quantisation of new indexer keys, then the paged write
+# ----------------------------------------------------------------------------
+#
+# "DeepSeek Sparse Attention DSA Architecture Guide", section "Stage 1: The
+# Lightning Indexer", item "Native FP8 Precision": indexer keys are stored as
+# 8-bit floats.  "Sparse Attention in Large Language Models: Architecture
+# Evolution and Engineering Practice", section 4, item "Memory Management and
+# KV Cache Optimization": the caches are paged.  "Sparse Attention
+# Architectures for Long-Context Inference: Evolution and Engineering
+# Practices", section 6, item "Incremental inference adaptation": every
+# decoding step writes the new tokens into the caches before attending.
+# The pages fix neither the scale rule nor the rounding; the reading taken
+# here is one fp32 scale per token, s = amax / 448 (1 when that is 0), and
+# code = E4M3(k / s) with k / s in fp32 and one round-to-nearest-even,
+# saturating at +-448.
+
+E4M3_MAX = 448.0          # largest finite E4M3 magnitude, 2^8 * (1 + 6/8)
+E4M3_MIN_EXP = 1 - E4M3_EXP_BIAS   # exponent of the smallest normal, -6
+E4M3_MANT_BITS = 3
+
+
+def e4m3_encode(y: np.ndarray) -> np.ndarray:
+    """OCP FP8 E4M3 code of each (finite) value: round to nearest, ties to
+    the even code, magnitudes above 448 saturate to 448; the sign bit is the
+    value's sign bit (so -0.0 and negatives that round to zero give 0x80).
+
+    In the binade [2^e, 2^(e+1)), e >= -6, the representable magnitudes are
+    the multiples of 2^(e-3); below 2^-6 (the subnormals) the multiples of
+    2^-9.  The nearest multiple is the rounded quotient, exact in float64.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    if not np.all(np.isfinite(y)):
+        raise ValueError("e4m3_encode: non-finite input")
+    a = np.abs(y)
+    _, ex = np.frexp(a)                         # a = m * 2^ex, m in [0.5, 1)
+    e = np.maximum(ex - 1, E4M3_MIN_EXP)        # floor(log2 a), clamped at the subnormals
+    quantum = np.ldexp(1.0, e - E4M3_MANT_BITS)
+    v = np.rint(a / quantum) * quantum          # np.rint: half to even
+    v = np.minimum(v, E4M3_MAX)
+    # code of the magnitude v
+    _, vex = np.frexp(v)
+    ve = vex - 1
+    normal = v >= 2.0 ** E4M3_MIN_EXP
+    e_field = np.where(normal, ve + E4M3_EXP_BIAS, 0)
+    mant = np.where(normal, v / np.ldexp(1.0, ve) - 1.0, v / 2.0 ** E4M3_MIN_EXP) * 8.0
+    mag = (e_field.astype(np.int64) << 3) | mant.astype(np.int64)
+    sign = np.signbit(y).astype(np.int64) << 7
+    return (sign | mag).astype(np.uint8)
+
+
+def quantise_keys(k: np.ndarray):
+    """Per-token FP8 quantisation of indexer keys k [n, d_I] (float32).
+
+    s[n] = fl32(amax_n / 448), replaced by 1 when it is 0 (an all-zero key, or
+    an amax so small that the quotient underflows); codes = E4M3(fl32(k / s)).
+    Returns (codes uint8 [n, d_I], s float32 [n]).  Non-finite keys raise.
+    """
+    k = np.asarray(k, dtype=np.float32)
+    if not np.all(np.isfinite(k)):
+        raise ValueError("quantise_keys: non-finite key")
+    amax = np.max(np.abs(k), axis=1) if k.shape[1] else np.zeros(k.shape[0], np.float32)
+    s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    y = (k / s[:, None]).astype(np.float32)
+    return e4m3_encode(y), s
+
+
+def append_destination(seq: int, pos: int, cache: dict, num_seqs: int, num_tokens: int):
+    """Physical row that token (seq, pos) is written to, or None when the
+    sequence, the position, the block-table slot or the page is out of range."""
+    if not (0 <= seq < num_seqs) or pos < 0:
+        return None
+    bt = cache.get("block_table")
+    if bt is not None:
+        page = int(cache["page_size"])
+        bt = np.asarray(bt)
+        if pos // page >= bt.shape[1]:
+            return None
+        p = int(bt[seq, pos // page])
+        if not (0 <= p < num_tokens // page):
+            return None
+    row = int(physical_rows(seq, np.array([pos]), cache)[0])
+    return row if 0 <= row < num_tokens else None
+
+
+def cache_append(inp: dict, num_seqs: int, tok_seq, tok_pos, k_new, latent_new):
+    """Write new tokens into copies of the caches of ``inp`` (num_seqs sequences).
+
+    Token n goes to physical row append_destination(tok_seq[n], tok_pos[n]):
+    its indexer key quantised by quantise_keys (e4m3 caches) or copied (f32
+    caches), its scale, and its latent row c || k^R copied bit for bit.  A
+    token whose destination is out of range, or whose key is not finite, is
+    not written and is listed in the returned ``bad`` set.  Destinations must
+    be distinct.  Returns (k_idx, k_scale, latent, bad).
+    """
+    k_idx = np.array(inp["k_idx"], copy=True)
+    k_scale = None if inp.get("k_scale") is None else np.array(inp["k_scale"], copy=True)
+    latent = np.array(inp["latent"], copy=True)
+    cache = inp["cache"]
+    num_tokens = latent.shape[0]
+    k_new = np.asarray(k_new, dtype=np.float32)
+    bad, seen = set(), set()
+    for n in range(len(tok_seq)):
+        row = append_destination(int(tok_seq[n]), int(tok_pos[n]), cache, num_seqs, num_tokens)
+        if row is None or not np.all(np.isfinite(k_new[n])):
+            bad.add(n)
+            continue
+        assert row not in seen, "two appended tokens share a destination"
+        seen.add(row)
+        if inp["idx_dtype"] == "e4m3":
+            codes, s = quantise_keys(k_new[n:n + 1])
+            k_idx[row] = codes[0]
+            k_scale[row] = s[0]
+        else:
+            k_idx[row] = k_new[n]
+        latent[row] = latent_new[n]
+    return k_idx, k_scale, latent, bad

@@ -272,3 +272,152 @@ def test_planted_keys_point_at_their_query():
             assert cos > 0.99 and abs(np.linalg.norm(kv) - 4 * math.sqrt(128)) < 2.0
             found += 1
     assert found > 0
+
+
+# --------------------------------------------------------------------------
+# P9: FP8 quantisation and the cache append
+# --------------------------------------------------------------------------
+
+_FINITE_CODES = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+
+
+def test_e4m3_encode_inverts_decode_on_every_finite_code():
+    # every representable value maps back to its own code, -0.0 included
+    assert np.array_equal(R.e4m3_encode(R.e4m3_decode(_FINITE_CODES)), _FINITE_CODES)
+
+
+def test_e4m3_encode_is_nearest_value_ties_to_even():
+    """Brute force over the 254 finite codes: the code of y is the one whose
+    value is nearest; of two equally near, the one with an even mantissa; above
+    448, the largest (saturation).  Ties are planted at every midpoint."""
+    vals = R.e4m3_decode(_FINITE_CODES)
+    pos = np.unique(vals[vals >= 0])
+    mids = (pos[1:] + pos[:-1]) / 2
+    rng = np.random.default_rng(7)
+    y = np.concatenate([mids, -mids, rng.uniform(-470, 470, 4000),
+                        rng.standard_normal(2000) * 2.0 ** rng.integers(-12, 6, 2000),
+                        [0.0, 448.0, 448.1, 463.9, 464.0, 1e30, -1e30]])
+    got = R.e4m3_encode(y)
+    for yi, g in zip(y, got):
+        d = np.abs(vals - min(abs(yi), 448.0) * (1 if yi >= 0 else -1))
+        cand = _FINITE_CODES[d == d.min()]
+        cand = cand[(cand >> 7) == (1 if np.signbit(yi) else 0)] if len(cand) > 1 else cand
+        if len(cand) > 1:
+            cand = cand[(cand & 1) == 0]
+        assert len(cand) == 1 and g == cand[0], (yi, hex(g), [hex(c) for c in cand])
+
+
+def test_e4m3_encode_matches_torch_cast_in_range():
+    # torch's float8 cast rounds to nearest even but turns overflow into NaN,
+    # so it is compared on [-448, 448]
+    import torch
+    rng = np.random.default_rng(8)
+    pos = np.unique(np.abs(R.e4m3_decode(_FINITE_CODES)))
+    mids = (pos[1:] + pos[:-1]) / 2                  # every tie, exact in fp32
+    y = np.concatenate([mids, -mids, rng.uniform(-448, 448, 20000),
+                        rng.standard_normal(20000) * 2.0 ** rng.integers(-14, 8, 20000)])
+    y = np.clip(y, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(R.e4m3_encode(y.astype(np.float64)), ref)
+
+
+def test_e4m3_encode_special_values():
+    cases = {448.0: 0x7E, 449.0: 0x7E, 1e9: 0x7E, -1e9: 0xFE, 2.0 ** -9: 0x01,
+             2.0 ** -10: 0x00, 3 * 2.0 ** -10: 0x02, 1.0: 0x38, -2.0: 0xC0, 0.0: 0x00,
+             1.0625: 0x38, 1.1875: 0x3A, 2.0 ** -6: 0x08, 7 * 2.0 ** -9: 0x07}
+    for y, c in cases.items():
+        assert R.e4m3_encode(np.array([y]))[0] == c, y
+    assert R.e4m3_encode(np.array([-0.0]))[0] == 0x80
+    assert R.e4m3_encode(np.array([-1e-6]))[0] == 0x80
+    with pytest.raises(ValueError):
+        R.e4m3_encode(np.array([np.nan]))
+
+
+def test_quantise_keys_error_bound_and_scale():
+    """Dequantised keys are within half a step of the input: relative 2^-4 in
+    the normal range, absolute 2^-10 * s below it; the largest magnitude of a
+    token lands on +-448; an all-zero token gets scale 1 and zero codes."""
+    rng = np.random.default_rng(9)
+    k = (rng.standard_normal((300, 128)) * np.exp(rng.uniform(-20, 8, (300, 1)))).astype(np.float32)
+    k[0] = 0.0
+    k[1, :] = 0.0
+    k[1, 5] = -3.0
+    codes, s = R.quantise_keys(k)
+    assert s.dtype == np.float32 and s[0] == 1.0 and not codes[0].any()
+    deq = R.e4m3_decode(codes) * s[:, None].astype(np.float64)
+    bound = np.maximum(2.0 ** -4 * np.abs(k.astype(np.float64)), 2.0 ** -10 * s[:, None])
+    assert np.all(np.abs(deq - k) <= bound * (1 + 1e-6))
+    assert np.all(np.abs(R.e4m3_decode(codes[1:])).max(axis=1) == 448.0)
+    assert codes[1, 5] == 0xFE and s[1] == np.float32(3.0) / np.float32(448)
+
+
+def test_quantise_keys_matches_generator_cast():
+    # the input generator quantises with torch's cast after a clip: another
+    # implementation of the same rule
+    rng = np.random.default_rng(10)
+    k = (rng.standard_normal((500, 128)) * 3).astype(np.float32)
+    codes, s = R.quantise_keys(k)
+    g_codes, g_s = I.to_e4m3_rows(k)
+    assert np.array_equal(codes, g_codes) and np.array_equal(s, g_s)
+
+
+def _logical_view(inp, seq, arr):
+    """A sequence's cache rows in logical order, built by concatenating its
+    pages in block-table order (paged) or slicing from its start."""
+    c = inp["cache"]
+    if c["block_table"] is not None:
+        pg = c["page_size"]
+        pages = [p for p in c["block_table"][seq] if p >= 0]
+        return np.concatenate([arr[p * pg:(p + 1) * pg] for p in pages])
+    return arr[int(c["seq_start"][seq]):]
+
+
+@pytest.mark.parametrize("paged", [True, False])
+def test_cache_append_writes_where_the_layout_says(paged):
+    cfg = I.CONFIGS["decode_128k_paged"].replace(ctx_lo=100, ctx_hi=300, n_seqs=3, paged=paged,
+                                                h_idx=2, d_idx=16, n_heads=2, d_c=8, d_r=8)
+    inp = I.generate(cfg, threads=1)
+    ctx = I.context_lengths(cfg)
+    rng = np.random.default_rng(11)
+    tok_seq = np.array([0, 2, 1, 2, 0, 1], dtype=np.int32)
+    tok_pos = np.array([0, int(ctx[2]) - 1, 65, 64, 63, int(ctx[1]) - 2], dtype=np.int32)
+    k_new = rng.standard_normal((6, 16)).astype(np.float32)
+    lat_new = rng.integers(0, 2 ** 15, (6, 16)).astype(np.uint16)
+    ki, ks, lat, bad = R.cache_append(inp, 3, tok_seq, tok_pos, k_new, lat_new)
+    assert bad == set()
+    codes, s = I.to_e4m3_rows(k_new)
+    written = set()
+    for n in range(6):
+        b, p = int(tok_seq[n]), int(tok_pos[n])
+        assert np.array_equal(_logical_view(inp, b, ki)[p], codes[n])
+        assert _logical_view(inp, b, ks)[p] == s[n]
+        assert np.array_equal(_logical_view(inp, b, lat)[p], lat_new[n])
+        written.add((b, p))
+    # every other row is untouched
+    changed = np.nonzero((ki != inp["k_idx"]).any(1) | (lat != inp["latent"]).any(1))[0]
+    assert len(changed) <= 6
+    for b in range(3):
+        v0, v1 = _logical_view(inp, b, inp["latent"]), _logical_view(inp, b, lat)
+        for p in range(int(ctx[b])):
+            if (b, p) not in written:
+                assert np.array_equal(v0[p], v1[p])
+
+
+def test_cache_append_rejects_out_of_range_and_non_finite():
+    cfg = I.CONFIGS["decode_128k_paged"].replace(ctx_lo=100, ctx_hi=130, n_seqs=2,
+                                                h_idx=2, d_idx=16, n_heads=2, d_c=8, d_r=8)
+    inp = I.generate(cfg, threads=1)
+    bt = inp["cache"]["block_table"]
+    bt[1, 1] = inp["cache"]["num_pages"]            # a page id past the pool
+    width = bt.shape[1] * 64
+    k_new = np.ones((8, 16), np.float32)
+    k_new[5, 3] = np.inf
+    lat_new = np.ones((8, 16), np.uint16)
+    # token:   0 ok, 1 seq<0, 2 seq>=2, 3 pos<0, 4 past the table, 5 inf key,
+    #          6 ok, 7 bad page id
+    tok_seq = [0, -1, 2, 1, 1, 1, 0, 1]
+    tok_pos = [3, 0, 0, -5, width, 7, 9, 70]
+    ki, ks, lat, bad = R.cache_append(inp, 2, tok_seq, tok_pos, k_new, lat_new)
+    assert bad == {1, 2, 3, 4, 5, 7}
+    changed = np.nonzero((ki != inp["k_idx"]).any(1) | (lat != inp["latent"]).any(1))[0]
+    assert sorted(changed) == sorted([bt[0, 0] * 64 + 3, bt[0, 0] * 64 + 9])

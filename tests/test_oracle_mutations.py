@@ -42,6 +42,54 @@ def _bad_e4m3_bias8(codes):
     return R_orig_e4m3(codes) / 2.0
 
 
+def _encode_variant(y, half_away=False, sat=448.0, min_exp=-6):
+    """The oracle's encoder with one slip switched on."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    _, ex = np.frexp(a)
+    e = np.maximum(ex - 1, min_exp)
+    quantum = np.ldexp(1.0, e - 3)
+    q = a / quantum
+    v = (np.floor(q + 0.5) if half_away else np.rint(q)) * quantum
+    v = np.minimum(v, sat)
+    _, vex = np.frexp(v)
+    ve = vex - 1
+    normal = v >= 2.0 ** min_exp
+    e_field = np.where(normal, ve + 7, 0)
+    mant = np.where(normal, v / np.ldexp(1.0, ve) - 1.0, v / 2.0 ** min_exp) * 8.0
+    mag = (e_field.astype(np.int64) << 3) | mant.astype(np.int64)
+    return ((np.signbit(y).astype(np.int64) << 7) | mag).astype(np.uint8)
+
+
+def _bad_encode_half_away(y):
+    return _encode_variant(y, half_away=True)
+
+
+def _bad_encode_no_saturation(y):
+    return _encode_variant(y, sat=480.0)
+
+
+def _bad_encode_subnormal_exponent(y):
+    return _encode_variant(y, min_exp=-7)
+
+
+def _bad_quantise_scale_240(k):
+    k = np.asarray(k, dtype=np.float32)
+    s = (np.max(np.abs(k), axis=1) / np.float32(240)).astype(np.float32)
+    s = np.where(s > 0, s, np.float32(1)).astype(np.float32)
+    return R.e4m3_encode((k / s[:, None]).astype(np.float32)), s
+
+
+def _bad_physical_rows_mirrored_offset(seq, s, cache):
+    s = np.asarray(s, dtype=np.int64)
+    bt = cache.get("block_table")
+    if bt is not None:
+        page = int(cache["page_size"])
+        return np.asarray(bt)[seq, s // page].astype(np.int64) * page + (page - 1 - s % page)
+    return R_orig_rows(seq, s, cache)
+
+
+R_orig_rows = R.physical_rows
 R_orig_mla = R.sparse_mla_row
 R_orig_e4m3 = R.e4m3_decode
 
@@ -54,6 +102,17 @@ CASES = [
     ("indexer_row", _bad_indexer_no_relu, [P.test_indexer_brute_force_fp8]),
     ("topk_row", _bad_topk_upper_tie, [P.test_topk_signed_zero_and_degenerate]),
     ("e4m3_decode", _bad_e4m3_bias8, [P.test_e4m3_decoder_matches_torch_on_all_codes]),
+    ("e4m3_encode", _bad_encode_half_away, [P.test_e4m3_encode_is_nearest_value_ties_to_even,
+                                            P.test_e4m3_encode_matches_torch_cast_in_range]),
+    ("e4m3_encode", _bad_encode_no_saturation, [P.test_e4m3_encode_special_values,
+                                                P.test_e4m3_encode_is_nearest_value_ties_to_even]),
+    ("e4m3_encode", _bad_encode_subnormal_exponent,
+     [P.test_e4m3_encode_inverts_decode_on_every_finite_code,
+      P.test_e4m3_encode_matches_torch_cast_in_range]),
+    ("quantise_keys", _bad_quantise_scale_240, [P.test_quantise_keys_error_bound_and_scale,
+                                                P.test_quantise_keys_matches_generator_cast]),
+    ("physical_rows", _bad_physical_rows_mirrored_offset,
+     [lambda: P.test_cache_append_writes_where_the_layout_says(True)]),
 ]
 
 
