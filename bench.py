@@ -18,6 +18,11 @@ ranks of the device time are the only cross-rank steps.
 
 `--impl reference` times the float64 CPU oracle (the only reference this
 method has) on a bounded sample of the same workload.
+
+`--op cache_append` measures the write that precedes the three stages
+instead: the workload's new tokens (a decode step's 32; all 65,536 of the 64K
+prefill, the default for this op) quantised to FP8 and written into the paged
+caches by one dsa_cache_append call.  Its metric is appended tokens/s.
 """
 from __future__ import annotations
 
@@ -44,7 +49,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode_128k_paged")
+    ap.add_argument("--workload", default=None,
+                    help="decode_128k_paged (path default) or prefill_64k (cache_append default)")
+    ap.add_argument("--op", default="path", choices=["path", "cache_append"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4, help="oracle rows per CPU-baseline sample")
@@ -472,8 +479,208 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- cache append
+APPEND_METRIC = "cache-append tokens/s (fused FP8 quantise + paged cache write)"
+APPEND_UNIT = "tokens/s"
+
+
+def append_bytes_per_token(cfg) -> int:
+    """Algorithmic bytes of one appended token: the fp32 key, the latent row,
+    its (seq, pos) and one block-table (or seq_start) entry read; the codes,
+    the scale and the latent row written."""
+    lat = cfg.d_qk * (2 if cfg.bf16 else 4)
+    key_in = 4 * cfg.d_idx
+    key_out = cfg.d_idx + 4 if cfg.fp8 else 4 * cfg.d_idx
+    return key_in + lat + 8 + 4 + key_out + lat
+
+
+def append_inputs(cfg):
+    from long_context_sparse_04_b200 import inputs as I
+    tok_seq, tok_pos = I.new_tokens(cfg)
+    k_new, lat_new = I.token_keys(cfg, tok_seq, tok_pos)
+    return tok_seq, tok_pos, k_new, lat_new
+
+
+def oracle_append_tokens_per_s(inp, cfg, toks, n):
+    from oracle import dsa_ref as R
+    tok_seq, tok_pos, k_new, lat_new = toks
+    c = inp["cache"]
+    num_seqs = c["block_table"].shape[0] if c["block_table"] is not None else len(c["seq_start"])
+    t0 = time.perf_counter()
+    R.cache_append(inp, num_seqs, tok_seq[:n], tok_pos[:n], k_new[:n], lat_new[:n])
+    dt = time.perf_counter() - t0
+    return n / dt, dt
+
+
+def run_append_reference(args, cfg):
+    from long_context_sparse_04_b200 import inputs as I
+    inp = I.generate(cfg, with_q=False)
+    toks = append_inputs(cfg)
+    n_tok = len(toks[0])
+    n = min(n_tok, 500)
+    for _ in range(args.warmup):
+        oracle_append_tokens_per_s(inp, cfg, toks, min(n, 16))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_append_tokens_per_s(inp, cfg, toks, n)
+    dt = time.perf_counter() - t0
+    value = args.steps * n / dt
+    line = {
+        "impl": "reference", "metric": APPEND_METRIC, "value": value, "unit": APPEND_UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 -> e4m3", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "tokens_per_step": n_tok},
+        "cpu_baseline": {"value": value, "unit": APPEND_UNIT, "cores": len(os.sched_getaffinity(0)),
+                         "kind": "oracle", "sample": f"{n} of {n_tok} tokens per step (NumPy)"},
+        "e2e": {"value": value, "unit": APPEND_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_append(args):
+    """One dsa_cache_append of the workload's new tokens per step."""
+    import torch
+    rank, world, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from long_context_sparse_04_b200 import build
+    build.build()
+    from long_context_sparse_04_b200 import _native as N
+    from long_context_sparse_04_b200 import inputs as I
+    from long_context_sparse_04_b200.workload import DeviceWorkload, to_device
+
+    cfg = I.CONFIGS[args.workload]
+    if args.n_seqs:
+        cfg = cfg.replace(n_seqs=args.n_seqs)
+    cfg_r = rank_config(cfg, rank)
+    inp = I.generate(cfg_r, with_q=False)
+    wl = DeviceWorkload(inp, device=dev)
+    toks = append_inputs(cfg_r)
+    n_tok = len(toks[0])
+    import numpy as np
+    d_in = [to_device(np.ascontiguousarray(toks[0], np.int32), dev),
+            to_device(np.ascontiguousarray(toks[1], np.int32), dev),
+            to_device(np.ascontiguousarray(toks[2], np.float32), dev), to_device(toks[3], dev)]
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step():
+        wl.append(*d_in)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = wl.status(N.DSA_OP_CACHE_APPEND)
+    assert st == (0, -1), f"device status {st}"
+    assert wl.kernels_ran(N.DSA_OP_CACHE_APPEND) & N.DSA_KERNEL_CACHE_APPEND
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    t_end = time.perf_counter() + 1.5
+    while time.perf_counter() < t_end:
+        for _ in range(20):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(ms), world, dev)
+    value = throughput(world, n_tok, args.steps, total_ms)
+
+    e2e = None
+    if not args.no_e2e:
+        host = [x.cpu().pin_memory() for x in d_in]
+        ws, ws_n = wl.workspace(N.DSA_OP_CACHE_APPEND)
+        host_st = torch.empty(8, dtype=torch.uint8).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in host)
+        tot = 0.0
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0.record(stream)
+            for d, h in zip(d_in, host):
+                d.copy_(h, non_blocking=True)
+            step()
+            host_st.copy_(ws[:8], non_blocking=True)   # the status word: the step's result
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                tot += e0.elapsed_time(e1)
+        tot = max_over_ranks(tot, world, dev)
+        e2e = {"value": throughput(world, n_tok, args.steps, tot), "unit": APPEND_UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 8}
+
+    peaks, peak_kind = measured_peaks()
+    avg_s = statistics.mean(ms) / 1e3
+    alg = append_bytes_per_token(cfg_r) * n_tok
+    achieved = alg / avg_s / 1e9
+    peak = peaks.get("hbm_gbs")
+    roof = {"kernel": "cache_append_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak if peak else None, "peak_source": peak_kind,
+            "traffic": kernel_traffic("cache_append_kernel", args.workload, alg),
+            "algorithmic_per_launch": alg}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        _, t1 = oracle_append_tokens_per_s(inp, cfg_r, toks, min(n_tok, 16))
+        n = int(max(1, min(n_tok, 16 * 10.0 / max(t1, 1e-4))))
+        v, dt = oracle_append_tokens_per_s(inp, cfg_r, toks, n)
+        cpu = {"value": v, "unit": APPEND_UNIT, "cores": len(os.sched_getaffinity(0)),
+               "kind": "oracle", "sample": f"{n} of {n_tok} tokens of one step, NumPy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": APPEND_METRIC, "value": value, "unit": APPEND_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 -> e4m3 (+ bf16 copy)", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "tokens_per_step": n_tok,
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "parallelism": f"{world} independent ranks (weak scaling)"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload is None:
+        args.workload = "prefill_64k" if args.op == "cache_append" else "decode_128k_paged"
+    if args.op == "cache_append":
+        if args.impl == "reference":
+            rank, _, _ = dist_info()
+            if rank != 0:
+                return 0
+            from long_context_sparse_04_b200 import inputs as I
+            return run_append_reference(args, I.CONFIGS[args.workload])
+        return run_append(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

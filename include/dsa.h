@@ -129,7 +129,8 @@ typedef enum {
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MLA = 2,
   DSA_OP_DECODE_STEP = 3,
-  DSA_OP_FORWARD = 4
+  DSA_OP_FORWARD = 4,
+  DSA_OP_CACHE_APPEND = 5
 } dsa_op;
 
 /* Human-readable name of a status code (static storage). */
@@ -143,7 +144,8 @@ int32_t dsa_version(void);
 
 /* Bytes of workspace `op` needs for these dimensions and rows (host only; it
  * reads the current device's SM count, which sets the decode key splits, and
- * uses 148 when no device is present).  Returns 0 for invalid arguments. */
+ * uses 148 when no device is present).  Returns 0 for invalid arguments.
+ * DSA_OP_CACHE_APPEND needs only the status block; `rows` may be NULL for it. */
 size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op);
 
 /* Zero the device status word at the head of `ws` (async on stream). */
@@ -163,6 +165,7 @@ dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status
 #define DSA_KERNEL_MLA_SIMT     0x08u
 #define DSA_KERNEL_MLA_TC       0x10u   /* tcgen05 bf16 sparse MLA */
 #define DSA_KERNEL_MLA_COMBINE  0x20u   /* split-K combine of the sparse MLA */
+#define DSA_KERNEL_CACHE_APPEND 0x40u   /* fused FP8 quantise + cache write */
 
 /* Synchronise `stream`, return the kernel trace of `ws` in *mask_out and clear it. */
 dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_out);
@@ -257,6 +260,47 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
                        const void* q_idx, const float* q_scale, const float* w,
                        const void* q, void* out, float* lse, int32_t* idx_out,
                        void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Cache append: the write that precedes the three stages of every decoding
+ * step ("Sparse Attention Architectures for Long-Context Inference: Evolution
+ * and Engineering Practices", section 6, item "Incremental inference
+ * adaptation": the caches are updated with each step's new tokens), into the
+ * paged caches of "Sparse Attention in Large Language Models: Architecture
+ * Evolution and Engineering Practice", section 4, item "Memory Management and
+ * KV Cache Optimization", with the indexer keys in FP8 ("DeepSeek Sparse
+ * Attention DSA Architecture Guide", section "Stage 1: The Lightning
+ * Indexer", item "Native FP8 Precision").  One kernel quantises and writes.
+ *
+ * Token n (0 <= n < n_new) goes to the physical row of logical position
+ * tok_pos[n] of sequence tok_seq[n], through the map every other call reads:
+ *   idx_k[row]       = E4M3(fl32(k_new[n, :] / s)),  s = fl32(amax_n / 448),
+ *                      s = 1 when that is 0; E4M3 rounds to nearest, ties to
+ *                      the even code, and saturates at +-448 (the OCP FP8
+ *                      encoding; -0.0 and negatives that round to 0 give 0x80)
+ *   idx_k_scale[row] = s
+ *   latent[row]      = latent_new[n, :]   (bit copy)
+ * With idx_dtype = DSA_F32 the key is copied and idx_k_scale is not used.
+ *   tok_seq, tok_pos [n_new] int32, device
+ *   k_new      [n_new, d_idx] fp32, device, 16-byte aligned; d_idx <= 512
+ *   latent_new [n_new, d_c + d_r] in mla_dtype, device, 16-byte aligned
+ * The caches that `cache` describes (latent, idx_k, idx_k_scale) are WRITTEN
+ * here and must be writable device memory; the descriptor's const qualifiers
+ * describe the other calls, which only read them.  Destinations must be
+ * distinct within one call (two tokens with one destination race).
+ * A token whose sequence is outside [0, num_seqs), whose position is negative
+ * or beyond the block table's width, whose block-table entry is outside
+ * [0, num_pages), or whose contiguous row is outside [0, num_tokens), is not
+ * written and is recorded in the device status word as DSA_ERR_OUT_OF_RANGE
+ * with detail n; a token whose key holds an infinity or NaN is not written
+ * either, and is recorded as DSA_ERR_INVALID_ARG with detail n (the first
+ * error of a launch wins).  The other tokens are written.
+ * ws: at least dsa_workspace_size(dims, NULL, DSA_OP_CACHE_APPEND) bytes (the
+ * status block), zeroed once by dsa_workspace_init.  n_new = 0 launches
+ * nothing. */
+dsa_status dsa_cache_append(const dsa_dims* dims, const dsa_cache* cache, int32_t n_new,
+                            const int32_t* tok_seq, const int32_t* tok_pos,
+                            const float* k_new, const void* latent_new,
+                            void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -15,8 +15,10 @@ DSA_ERR_OUT_OF_RANGE, DSA_ERR_TIMEOUT, DSA_ERR_WORKSPACE = 4, 5, 6
 DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
 DSA_ALGO_AUTO, DSA_ALGO_SIMT = 0, 1
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE_STEP, DSA_OP_FORWARD = range(5)
+DSA_OP_CACHE_APPEND = 5
 DSA_KERNEL_INDEXER_SIMT, DSA_KERNEL_INDEXER_TC, DSA_KERNEL_TOPK = 0x01, 0x02, 0x04
 DSA_KERNEL_MLA_SIMT, DSA_KERNEL_MLA_TC, DSA_KERNEL_MLA_COMBINE = 0x08, 0x10, 0x20
+DSA_KERNEL_CACHE_APPEND = 0x40
 
 
 class dsa_dims(ctypes.Structure):
@@ -60,6 +62,8 @@ _SIGS = {
                                        ctypes.c_size_t, _P]),
     "dsa_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                    ctypes.c_size_t, _P]),
+    "dsa_cache_append": (ctypes.c_int, [_P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]),
 }
 
 
@@ -156,3 +160,9 @@ def dsa_forward(dims, rows, cache, q_idx, q_scale, w, q, out, lse, idx_out, ws, 
                 stream, check=True):
     return _call("dsa_forward", _ref(dims), _ref(rows), _ref(cache), q_idx, q_scale, w, q, out,
                  lse, idx_out, ws, ws_bytes, stream, check=check)
+
+
+def dsa_cache_append(dims, cache, n_new, tok_seq, tok_pos, k_new, latent_new, ws, ws_bytes,
+                     stream, check=True):
+    return _call("dsa_cache_append", _ref(dims), _ref(cache), n_new, tok_seq, tok_pos, k_new,
+                 latent_new, ws, ws_bytes, stream, check=check)

@@ -324,6 +324,7 @@ const char* dsa_last_error(void) { return g_err; }
 int32_t dsa_version(void) { return 100; }
 
 size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op) {
+  if (op == DSA_OP_CACHE_APPEND) return check_dims(dims) == DSA_OK ? kStatusBytes : 0;
   if (check_dims(dims) != DSA_OK || check_rows(rows) != DSA_OK) return 0;
   if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
   return plan(dims, rows, op).total;
@@ -583,6 +584,43 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     if ((st = run_mla(dims, ma, s))) return st;
   }
   return DSA_OK;
+}
+
+dsa_status dsa_cache_append(const dsa_dims* dims, const dsa_cache* cache, int32_t n_new,
+                            const int32_t* tok_seq, const int32_t* tok_pos,
+                            const float* k_new, const void* latent_new,
+                            void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) != DSA_OK) return st;
+  if ((st = check_cache(cache, dims, true, true)) != DSA_OK) return st;
+  CHECK_ARG(n_new >= 0, "n_new must be >= 0");
+  if ((st = check_ws(ws, ws_bytes, kStatusBytes)) != DSA_OK) return st;
+  if (dims->d_idx > cache_append_max_d_idx()) {
+    set_error("cache append takes d_idx <= %d", cache_append_max_d_idx());
+    return DSA_ERR_UNSUPPORTED;
+  }
+  if (n_new == 0) return DSA_OK;
+  CHECK_ARG(tok_seq != nullptr && tok_pos != nullptr, "tok_seq / tok_pos is NULL");
+  CHECK_ARG(k_new != nullptr && aligned(k_new, 16), "k_new must be non-NULL and 16-byte aligned");
+  CHECK_ARG(latent_new != nullptr && aligned(latent_new, 16),
+            "latent_new must be non-NULL and 16-byte aligned");
+  AppendArgs a{};
+  a.n_new = n_new;
+  a.tok_seq = tok_seq;
+  a.tok_pos = tok_pos;
+  a.k_new = k_new;
+  a.latent_new = latent_new;
+  a.d_idx = dims->d_idx;
+  a.latent_row_bytes = (dims->d_c + dims->d_r) * (dims->mla_dtype == DSA_BF16 ? 2 : 4);
+  a.idx_dtype = dims->idx_dtype;
+  // the caches are written here; the descriptor is shared with the read-only calls
+  a.idx_k = const_cast<void*>(cache->idx_k);
+  a.idx_k_scale = const_cast<float*>(cache->idx_k_scale);
+  a.latent = const_cast<void*>(cache->latent);
+  a.map = make_map(cache);
+  a.num_seqs = cache->num_seqs;
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  return launch_cache_append(a, (cudaStream_t)stream);
 }
 
 }  // extern "C"

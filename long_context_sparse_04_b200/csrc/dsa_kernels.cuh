@@ -58,6 +58,23 @@ struct MlaArgs {
   long long* trace;           // profiling stamps or null
 };
 
+struct AppendArgs {
+  int n_new;
+  const int32_t* tok_seq;     // [n_new]
+  const int32_t* tok_pos;     // [n_new]
+  const float* k_new;         // [n_new, d_I] fp32
+  const void* latent_new;     // [n_new, d_c + d_r] in the latent cache's dtype
+  int d_idx;
+  int latent_row_bytes;       // (d_c + d_r) * element size, a multiple of 16
+  dsa_dtype idx_dtype;
+  void* idx_k;                // written: [num_tokens, d_I] e4m3 | f32
+  float* idx_k_scale;         // written: [num_tokens] (e4m3 only)
+  void* latent;               // written: [num_tokens, d_c + d_r]
+  CacheMap map;
+  int num_seqs;
+  DeviceStatus* status;
+};
+
 // Profiling trace buffer registered on the calling host thread (or null).
 long long* trace_buffer();
 static constexpr int kTraceEvents = 8, kTraceBlocks = 32;
@@ -76,6 +93,9 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream);
 bool mla_tc_supported(const MlaArgs& a);
 int mla_tc_splits(int num_rows);
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
+
+dsa_status launch_cache_append(const AppendArgs& a, cudaStream_t stream);
+int cache_append_max_d_idx();
 
 // Per-device host state.  Kernel attributes and device properties belong to a
 // device, so a process that drives several GPUs sets and caches them per

@@ -167,3 +167,20 @@ class DeviceWorkload:
                       _vp(self.w), _vp(self.q), _vp(out), _vp(lse), _vp(idx), _vp(ws), n,
                       self.stream)
         return out, lse, idx
+
+    def append(self, tok_seq, tok_pos, k_new, latent_new, check=True):
+        """dsa_cache_append of new tokens (device tensors: int32 [n], int32 [n],
+        fp32 [n, d_I], latent rows [n, d_c+d_r]) into this workload's caches."""
+        ws, n = self.workspace(N.DSA_OP_CACHE_APPEND)
+        return N.dsa_cache_append(self.dims, self.cache, int(tok_seq.shape[0]), _vp(tok_seq),
+                                  _vp(tok_pos), _vp(k_new), _vp(latent_new), _vp(ws), n,
+                                  self.stream, check=check)
+
+    def caches_to_host(self):
+        """(k_idx, k_scale, latent) in their storage formats (bf16 as uint16 bits)."""
+        torch = self.torch
+        lat = self.latent
+        lat = lat.view(torch.int16).cpu().numpy().view(np.uint16) if lat.dtype == torch.bfloat16 \
+            else lat.cpu().numpy()
+        ks = None if self.k_scale is None else self.k_scale.cpu().numpy()
+        return self.k_idx.cpu().numpy(), ks, lat
