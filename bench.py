@@ -514,7 +514,7 @@ def oracle_append_tokens_per_s(inp, cfg, toks, n):
 
 def run_append_reference(args, cfg):
     from long_context_sparse_04_b200 import inputs as I
-    inp = I.generate(cfg, with_q=False)
+    inp = I.generate(cfg, with_q=False, rows=[])       # the caches only
     toks = append_inputs(cfg)
     n_tok = len(toks[0])
     n = min(n_tok, 500)
@@ -541,6 +541,7 @@ def run_append_reference(args, cfg):
 
 def run_append(args):
     """One dsa_cache_append of the workload's new tokens per step."""
+    import numpy as np
     import torch
     rank, world, local = dist_info()
     if world > 1:
@@ -560,11 +561,10 @@ def run_append(args):
     if args.n_seqs:
         cfg = cfg.replace(n_seqs=args.n_seqs)
     cfg_r = rank_config(cfg, rank)
-    inp = I.generate(cfg_r, with_q=False)
+    inp = I.generate(cfg_r, with_q=False, rows=[])     # the caches only
     wl = DeviceWorkload(inp, device=dev)
     toks = append_inputs(cfg_r)
     n_tok = len(toks[0])
-    import numpy as np
     d_in = [to_device(np.ascontiguousarray(toks[0], np.int32), dev),
             to_device(np.ascontiguousarray(toks[1], np.int32), dev),
             to_device(np.ascontiguousarray(toks[2], np.float32), dev), to_device(toks[3], dev)]

@@ -153,6 +153,8 @@ def qidx_rows_f32(cfg: DSAConfig, rows) -> np.ndarray:
 
 
 def w_rows(cfg: DSAConfig, rows) -> np.ndarray:
+    if len(rows) == 0:
+        return np.zeros((0, cfg.h_idx), np.float32)
     return np.stack([_normal(cfg.seed, TID_W, (int(t),), (cfg.h_idx,), cfg.std_w) for t in rows])
 
 
