@@ -38,6 +38,10 @@ section and equation on that page):
   token (an encoder written from the OCP definition: nearest value, ties to
   the even code, saturating at +-448) and written with their latent rows at
   the rows the block table gives.
+* same section, output equation, with the page's "End-to-End Implementation"
+  module: the output projection after the path, u_{t,i} = W_UV,i o_{t,i} per
+  head (W_UV,i is constant in s, so it moves out of the softmax sum) and
+  y_t = W_out [u_{t,1}; ...; u_{t,H}].
 * section "The Classical Multi-Head Latent Attention (MLA) Mechanism", logit
   equation A_{t,s,i}: the dense MLA that sparse MLA must equal when k covers
   every visible key, and the un-absorbed form used for the absorbed ==
@@ -397,3 +401,24 @@ def cache_append(inp: dict, num_seqs: int, tok_seq, tok_pos, k_new, latent_new):
             k_idx[row] = k_new[n]
         latent[row] = latent_new[n]
     return k_idx, k_scale, latent, bad
+
+
+# ----------------------------------------------------------------------------
+# Output projection: W_UV per head, then W_out over the concatenated heads
+# ----------------------------------------------------------------------------
+#
+# "DeepSeek Sparse Attention DSA Architecture Guide", section "Stage 2:
+# Fine-Grained Token Selection and Output Computation", output equation:
+# u_{t,i} = sum_s softmax_s(.) W_{UV,i} c_s.  W_{UV,i} does not depend on s, so
+# u_{t,i} = W_{UV,i} o_{t,i} with o_{t,i} = sum_s softmax_s(.) c_s, the latent
+# output of the sparse attention.  The page's module ("End-to-End
+# Implementation") then concatenates the heads in head order and applies its
+# output projection w_out.
+
+def output_projection_row(o: np.ndarray, w_uv: np.ndarray, w_out: np.ndarray):
+    """o [H, d_c], w_uv [H, d_v, d_c], w_out [d_model, H*d_v] (float64).
+    u[i] = W_UV[i] @ o[i];  y = W_out @ [u[0]; u[1]; ...; u[H-1]].
+    Returns (u [H, d_v], y [d_model])."""
+    u = np.einsum("ivc,ic->iv", w_uv, o)
+    y = w_out @ u.reshape(-1)
+    return u, y

@@ -421,3 +421,49 @@ def test_cache_append_rejects_out_of_range_and_non_finite():
     assert bad == {1, 2, 3, 4, 5, 7}
     changed = np.nonzero((ki != inp["k_idx"]).any(1) | (lat != inp["latent"]).any(1))[0]
     assert sorted(changed) == sorted([bt[0, 0] * 64 + 3, bt[0, 0] * 64 + 9])
+
+
+# --------------------------------------------------------------------------
+# P10: the output projection (W_UV per head, then W_out)
+# --------------------------------------------------------------------------
+
+def test_output_projection_brute_force():
+    """Scalar loops over the definition: u[i][v] = sum_c W_UV[i][v][c] o[i][c],
+    y[m] = sum_i sum_v W_out[m][i*d_v + v] u[i][v]."""
+    rng = np.random.default_rng(20)
+    H, d_c, d_v, d_model = 3, 5, 4, 6
+    o = rng.standard_normal((H, d_c))
+    w_uv = rng.standard_normal((H, d_v, d_c))
+    w_out = rng.standard_normal((d_model, H * d_v))
+    u_ref = [[sum(w_uv[i][v][c] * o[i][c] for c in range(d_c)) for v in range(d_v)] for i in range(H)]
+    y_ref = [sum(w_out[m][i * d_v + v] * u_ref[i][v] for i in range(H) for v in range(d_v))
+             for m in range(d_model)]
+    u, y = R.output_projection_row(o, w_uv, w_out)
+    np.testing.assert_allclose(u, np.array(u_ref), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(y, np.array(y_ref), rtol=1e-13, atol=1e-13)
+
+
+def test_output_projection_completes_the_pages_module():
+    """The page's module: values uncompressed per selected row by one linear
+    layer (H*d_v outputs, viewed as [H, d_v]), weighted by the softmax, heads
+    concatenated in order, then the output linear layer; written with torch
+    library routines.  The oracle's path (sparse MLA latent output, then the
+    projection) must give the same y."""
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(21)
+    H, d_c, d_r, d_v, d_model, n = 4, 12, 6, 5, 7, 9
+    q = rng.standard_normal((H, d_c + d_r)) * 0.3
+    kv = rng.standard_normal((n, d_c + d_r))
+    w_uv = rng.standard_normal((H, d_v, d_c))
+    w_out = rng.standard_normal((d_model, H * d_v))
+    sm = 1 / math.sqrt(d_c + d_r)
+    o, _ = R.sparse_mla_row(q, kv, d_c, sm)
+    _, y = R.output_projection_row(o, w_uv, w_out)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    c = t(kv[:, :d_c])
+    p = torch.softmax(t(q) @ t(kv).T * sm, dim=-1)                   # [H, n]
+    v = F.linear(c, t(w_uv.reshape(H * d_v, d_c))).view(n, H, d_v)    # per selected row
+    attn = torch.einsum("is,siv->iv", p, v).reshape(H * d_v)
+    y_page = F.linear(attn, t(w_out)).numpy()
+    np.testing.assert_allclose(y, y_page, rtol=1e-11, atol=1e-12)

@@ -89,6 +89,16 @@ def _bad_physical_rows_mirrored_offset(seq, s, cache):
     return R_orig_rows(seq, s, cache)
 
 
+def _bad_outproj_dim_major(o, w_uv, w_out):
+    u = np.einsum("ivc,ic->iv", w_uv, o)
+    return u, w_out @ u.T.reshape(-1)
+
+
+def _bad_outproj_head0_weights(o, w_uv, w_out):
+    u = np.einsum("vc,ic->iv", w_uv[0], o)
+    return u, w_out @ u.reshape(-1)
+
+
 R_orig_rows = R.physical_rows
 R_orig_mla = R.sparse_mla_row
 R_orig_e4m3 = R.e4m3_decode
@@ -111,6 +121,10 @@ CASES = [
       P.test_e4m3_encode_matches_torch_cast_in_range]),
     ("quantise_keys", _bad_quantise_scale_240, [P.test_quantise_keys_error_bound_and_scale,
                                                 P.test_quantise_keys_matches_generator_cast]),
+    ("output_projection_row", _bad_outproj_dim_major,
+     [P.test_output_projection_brute_force, P.test_output_projection_completes_the_pages_module]),
+    ("output_projection_row", _bad_outproj_head0_weights,
+     [P.test_output_projection_brute_force, P.test_output_projection_completes_the_pages_module]),
     ("physical_rows", _bad_physical_rows_mirrored_offset,
      [lambda: P.test_cache_append_writes_where_the_layout_says(True)]),
 ]
