@@ -23,6 +23,11 @@ method has) on a bounded sample of the same workload.
 instead: the workload's new tokens (a decode step's 32; all 65,536 of the 64K
 prefill, the default for this op) quantised to FP8 and written into the paged
 caches by one dsa_cache_append call.  Its metric is appended tokens/s.
+
+`--op output_projection` measures the two GEMMs after the path (u = W_UV o
+per head, y = W_out u) for the workload's query rows (32 in decode, 65,536 in
+the 64K prefill) with H = 128, d_c = 512, d_v = 128, d_model = 7168: one
+dsa_output_projection call per step.  Its metric is rows/s.
 """
 from __future__ import annotations
 
@@ -51,7 +56,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=None,
                     help="decode_128k_paged (path default) or prefill_64k (cache_append default)")
-    ap.add_argument("--op", default="path", choices=["path", "cache_append"])
+    ap.add_argument("--op", default="path", choices=["path", "cache_append", "output_projection"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4, help="oracle rows per CPU-baseline sample")
@@ -669,10 +674,209 @@ def run_append(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- output projection
+PROJ_METRIC = "output-projection rows/s (u = W_UV o per head, y = W_out u)"
+PROJ_UNIT = "rows/s"
+
+
+def proj_algorithmic(cfg, T):
+    """FLOPs and minimum HBM bytes of one dsa_output_projection call: both
+    weight matrices read once, o read, u written and read back, y written."""
+    H, d_c, d_v, dm = cfg.n_heads, cfg.d_c, cfg.d_v, cfg.d_model
+    flops = 2 * T * H * d_v * (d_c + dm)
+    by = 2 * (H * d_v * d_c + dm * H * d_v) + 2 * T * (H * d_c + 2 * H * d_v + dm)
+    return flops, by
+
+
+def oracle_proj_rows_per_s(o_bits, w_uv, w_out, rows):
+    from oracle import dsa_ref as R
+    wu, wo = R.bf16_decode(w_uv), R.bf16_decode(w_out)
+    t0 = time.perf_counter()
+    for t in rows:
+        R.output_projection_row(R.bf16_decode(o_bits[t]), wu, wo)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, dt
+
+
+def run_out_proj(args):
+    import ctypes
+    import numpy as np
+    import torch
+    rank, world, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from long_context_sparse_04_b200 import build
+    build.build()
+    from long_context_sparse_04_b200 import _native as N
+    from long_context_sparse_04_b200 import inputs as I
+    from long_context_sparse_04_b200.workload import to_device
+
+    cfg = rank_config(I.CONFIGS[args.workload], rank)
+    T = cfg.n_rows
+    w_uv_h, w_out_h = I.out_proj_weights(cfg)
+    blk = min(T, 1024)
+    o_blk = I.latent_out_rows(cfg, range(blk))
+    o = to_device(o_blk, dev).repeat((T + blk - 1) // blk, 1, 1)[:T].contiguous()
+    w_uv, w_out = to_device(w_uv_h, dev), to_device(w_out_h, dev)
+    u = torch.empty((T, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T, cfg.d_model), dtype=torch.bfloat16, device=dev)
+    dims = N.dsa_proj_dims(n_heads=cfg.n_heads, d_c=cfg.d_c, d_v=cfg.d_v, d_model=cfg.d_model)
+    nbytes = N.dsa_output_projection_ws_size(dims, T)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = lambda x: ctypes.c_void_p(x.data_ptr())
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step():
+        N.dsa_output_projection(dims, T, vp(o), vp(w_uv), vp(w_out), vp(u), vp(y), vp(ws), nbytes, sp)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = N.dsa_read_device_status(vp(ws), sp)
+    assert st == (0, -1), f"device status {st}"
+    ran = N.dsa_read_kernel_trace(vp(ws), sp)
+    assert ran & N.DSA_KERNEL_OUT_PROJ
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    t_end = time.perf_counter() + 1.5
+    while time.perf_counter() < t_end:
+        for _ in range(20 if T < 4096 else 1):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append(e0.elapsed_time(e1))
+    barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(ms), world, dev)
+    value = throughput(world, T, args.steps, total_ms)
+    launches = 2 + (1 if ran & N.DSA_KERNEL_OUT_PROJ_REDUCE else 0)
+
+    e2e = None
+    if not args.no_e2e and T * cfg.n_heads * cfg.d_c * 2 <= (1 << 30):
+        host_o = o.cpu().pin_memory()
+        host_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        tot = 0.0
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0.record(stream)
+            o.copy_(host_o, non_blocking=True)
+            step()
+            host_y.copy_(y, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                tot += e0.elapsed_time(e1)
+        tot = max_over_ranks(tot, world, dev)
+        e2e = {"value": throughput(world, T, args.steps, tot), "unit": PROJ_UNIT,
+               "h2d_bytes_per_step": host_o.numel() * 2, "d2h_bytes_per_step": host_y.numel() * 2}
+
+    peaks, peak_kind = measured_peaks()
+    avg_s = statistics.mean(ms) / 1e3
+    flops, by = proj_algorithmic(cfg, T)
+    if T >= 4096:      # the products are tensor-bound at prefill batch sizes
+        roof = {"kernel": "out_proj_kernel (both launches)", "bound": "tensor",
+                "achieved": flops / avg_s / 1e12, "peak": peaks.get("bf16_tflops"), "unit": "TFLOP/s",
+                "algorithmic_per_launch": flops}
+    else:              # decode: the weights' HBM stream
+        roof = {"kernel": "out_proj_kernel (both launches)", "bound": "hbm",
+                "achieved": by / avg_s / 1e9, "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
+                "algorithmic_per_launch": by}
+    roof["frac"] = roof["achieved"] / roof["peak"] if roof["peak"] else None
+    roof["peak_source"] = peak_kind
+    roof["traffic"] = kernel_traffic("out_proj_kernel", args.workload, by)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        _, t1 = oracle_proj_rows_per_s(o_blk, w_uv_h, w_out_h, [0])
+        n = int(max(1, min(blk, 10.0 / max(t1, 1e-3))))
+        v, dt = oracle_proj_rows_per_s(o_blk, w_uv_h, w_out_h, list(range(n)))
+        cpu = {"value": v, "unit": PROJ_UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"{n} of {T} rows, float64 NumPy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": PROJ_METRIC, "value": value, "unit": PROJ_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: {T} rows, H={cfg.n_heads} d_c={cfg.d_c} "
+                                   f"d_v={cfg.d_v} d_model={cfg.d_model}; o is a seeded "
+                                   f"{blk}-row block repeated down the rows",
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "parallelism": f"{world} independent ranks (weak scaling)"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_out_proj_reference(args, cfg):
+    from long_context_sparse_04_b200 import inputs as I
+    T = cfg.n_rows
+    w_uv, w_out = I.out_proj_weights(cfg)
+    o = I.latent_out_rows(cfg, range(min(T, 4)))
+    for _ in range(args.warmup):
+        oracle_proj_rows_per_s(o, w_uv, w_out, [0])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_proj_rows_per_s(o, w_uv, w_out, list(range(len(o))))
+    dt = time.perf_counter() - t0
+    value = args.steps * len(o) / dt
+    line = {
+        "impl": "reference", "metric": PROJ_METRIC, "value": value, "unit": PROJ_UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {T} rows, H={cfg.n_heads} d_c={cfg.d_c} "
+                               f"d_v={cfg.d_v} d_model={cfg.d_model}"},
+        "cpu_baseline": {"value": value, "unit": PROJ_UNIT, "cores": len(os.sched_getaffinity(0)),
+                         "kind": "oracle", "sample": f"{len(o)} of {T} rows per step (float64 NumPy)"},
+        "e2e": {"value": value, "unit": PROJ_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.workload is None:
-        args.workload = "prefill_64k" if args.op == "cache_append" else "decode_128k_paged"
+        args.workload = "prefill_64k" if args.op in ("cache_append", "output_projection") \
+            else "decode_128k_paged"
+    if args.op == "output_projection":
+        if args.impl == "reference":
+            rank, _, _ = dist_info()
+            if rank != 0:
+                return 0
+            from long_context_sparse_04_b200 import inputs as I
+            return run_out_proj_reference(args, I.CONFIGS[args.workload])
+        return run_out_proj(args)
     if args.op == "cache_append":
         if args.impl == "reference":
             rank, _, _ = dist_info()

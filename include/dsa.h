@@ -166,6 +166,8 @@ dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status
 #define DSA_KERNEL_MLA_TC       0x10u   /* tcgen05 bf16 sparse MLA */
 #define DSA_KERNEL_MLA_COMBINE  0x20u   /* split-K combine of the sparse MLA */
 #define DSA_KERNEL_CACHE_APPEND 0x40u   /* fused FP8 quantise + cache write */
+#define DSA_KERNEL_OUT_PROJ     0x80u   /* tcgen05 output projection GEMM */
+#define DSA_KERNEL_OUT_PROJ_REDUCE 0x100u   /* split-K sum of the W_out product */
 
 /* Synchronise `stream`, return the kernel trace of `ws` in *mask_out and clear it. */
 dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_out);
@@ -301,6 +303,43 @@ dsa_status dsa_cache_append(const dsa_dims* dims, const dsa_cache* cache, int32_
                             const int32_t* tok_seq, const int32_t* tok_pos,
                             const float* k_new, const void* latent_new,
                             void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Output projection: the two GEMMs after the path that complete u_t
+ * ("DeepSeek Sparse Attention DSA Architecture Guide", section "Stage 2:
+ * Fine-Grained Token Selection and Output Computation", output equation
+ * u_{t,i} = sum_s softmax_s(.) W_{UV,i} c_s; W_{UV,i} does not depend on s, so
+ * it applies once to the latent output o of dsa_sparse_mla_fwd; then the
+ * output projection of the page's module, "End-to-End Implementation", over
+ * the heads concatenated in order):
+ *     u[t,i,:] = W_UV[i] o[t,i,:]                     (i < H)
+ *     y[t,:]   = W_out [u[t,0,:]; u[t,1,:]; ...; u[t,H-1,:]]
+ * bf16 operands, fp32 accumulation on the tensor cores; u is rounded to bf16
+ * once and y is computed from that bf16 u, then rounded to bf16 once (a K
+ * split adds its fp32 partials in a fixed order first). */
+typedef struct {
+  int32_t n_heads;   /* H                                                        */
+  int32_t d_c;       /* latent width per head (the attention output), a multiple of 64 */
+  int32_t d_v;       /* value head width after W_UV: a multiple of 32, at most 256,
+                        with H * d_v a multiple of 64                             */
+  int32_t d_model;   /* output width after W_out, a multiple of 32               */
+} dsa_proj_dims;
+
+/* Workspace bytes of dsa_output_projection for num_rows rows (host only; it
+ * reads the current device's SM count, which sets the K splits of small
+ * batches).  Returns 0 for invalid dimensions. */
+size_t dsa_output_projection_ws_size(const dsa_proj_dims* dims, int32_t num_rows);
+
+/*   o     [T, H, d_c] bf16: the latent attention output (dsa_sparse_mla_fwd's out)
+ *   w_uv  [H, d_v, d_c] bf16, row-major: W_UV[i] is a d_v x d_c matrix
+ *   w_out [d_model, H*d_v] bf16, row-major: column i*d_v + v multiplies u[t,i,v]
+ *   u     [T, H, d_v] bf16 out (the per-head values, kept for the caller)
+ *   y     [T, d_model] bf16 out
+ * All device pointers, 16-byte aligned, owned by the caller; u and y must not
+ * overlap the inputs.  ws: dsa_output_projection_ws_size bytes, 256-byte
+ * aligned (status block, then split-K partials).  T = 0 launches nothing. */
+dsa_status dsa_output_projection(const dsa_proj_dims* dims, int32_t num_rows, const void* o,
+                                 const void* w_uv, const void* w_out, void* u, void* y,
+                                 void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,6 +19,7 @@ DSA_OP_CACHE_APPEND = 5
 DSA_KERNEL_INDEXER_SIMT, DSA_KERNEL_INDEXER_TC, DSA_KERNEL_TOPK = 0x01, 0x02, 0x04
 DSA_KERNEL_MLA_SIMT, DSA_KERNEL_MLA_TC, DSA_KERNEL_MLA_COMBINE = 0x08, 0x10, 0x20
 DSA_KERNEL_CACHE_APPEND = 0x40
+DSA_KERNEL_OUT_PROJ, DSA_KERNEL_OUT_PROJ_REDUCE = 0x80, 0x100
 
 
 class dsa_dims(ctypes.Structure):
@@ -40,6 +41,11 @@ class dsa_cache(ctypes.Structure):
                 ("block_table", ctypes.c_void_p), ("page_size", ctypes.c_int32),
                 ("max_pages_per_seq", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
                 ("num_tokens", ctypes.c_int64)]
+
+
+class dsa_proj_dims(ctypes.Structure):
+    _fields_ = [("n_heads", ctypes.c_int32), ("d_c", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("d_model", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -64,6 +70,9 @@ _SIGS = {
                                    ctypes.c_size_t, _P]),
     "dsa_cache_append": (ctypes.c_int, [_P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
+    "dsa_output_projection_ws_size": (ctypes.c_size_t, [_P, ctypes.c_int32]),
+    "dsa_output_projection": (ctypes.c_int, [_P, ctypes.c_int32, _P, _P, _P, _P, _P, _P,
+                                             ctypes.c_size_t, _P]),
 }
 
 
@@ -166,3 +175,12 @@ def dsa_cache_append(dims, cache, n_new, tok_seq, tok_pos, k_new, latent_new, ws
                      stream, check=True):
     return _call("dsa_cache_append", _ref(dims), _ref(cache), n_new, tok_seq, tok_pos, k_new,
                  latent_new, ws, ws_bytes, stream, check=check)
+
+
+def dsa_output_projection_ws_size(dims, num_rows) -> int:
+    return LIB.dsa_output_projection_ws_size(_ref(dims), num_rows)
+
+
+def dsa_output_projection(dims, num_rows, o, w_uv, w_out, u, y, ws, ws_bytes, stream, check=True):
+    return _call("dsa_output_projection", _ref(dims), num_rows, o, w_uv, w_out, u, y, ws, ws_bytes,
+                 stream, check=check)

@@ -124,6 +124,23 @@ dsa_status check_cache(const dsa_cache* c, const dsa_dims* d, bool need_idx, boo
   return DSA_OK;
 }
 
+dsa_status check_proj(const dsa_proj_dims* d) {
+  CHECK_ARG(d != nullptr, "dims is NULL");
+  CHECK_ARG(d->n_heads > 0 && d->d_c > 0 && d->d_v > 0 && d->d_model > 0, "non-positive dimension");
+  if (d->d_c % 64 != 0 || d->d_v % 32 != 0 || d->d_v > 256 || (d->n_heads * d->d_v) % 64 != 0 ||
+      d->d_model % 32 != 0) {
+    set_error("output projection takes d_c %% 64 == 0, d_v %% 32 == 0, d_v <= 256, "
+              "H*d_v %% 64 == 0, d_model %% 32 == 0");
+    return DSA_ERR_UNSUPPORTED;
+  }
+  return DSA_OK;
+}
+
+size_t proj_partial_bytes(const dsa_proj_dims* d, int32_t T) {
+  const int splits = out_proj_splits(T, d->d_model, d->n_heads * d->d_v / 64);
+  return splits > 1 ? align_up((size_t)splits * (size_t)T * (size_t)d->d_model * sizeof(float)) : 0;
+}
+
 CacheMap make_map(const dsa_cache* c) {
   CacheMap m{};
   m.seq_start = c->seq_start;
@@ -621,6 +638,44 @@ dsa_status dsa_cache_append(const dsa_dims* dims, const dsa_cache* cache, int32_
   a.num_seqs = cache->num_seqs;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
   return launch_cache_append(a, (cudaStream_t)stream);
+}
+
+size_t dsa_output_projection_ws_size(const dsa_proj_dims* dims, int32_t num_rows) {
+  if (check_proj(dims) != DSA_OK || num_rows < 0) return 0;
+  return kStatusBytes + proj_partial_bytes(dims, num_rows);
+}
+
+dsa_status dsa_output_projection(const dsa_proj_dims* dims, int32_t num_rows, const void* o,
+                                 const void* w_uv, const void* w_out, void* u, void* y,
+                                 void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_proj(dims)) != DSA_OK) return st;
+  CHECK_ARG(num_rows >= 0, "num_rows must be >= 0");
+  if ((st = check_ws(ws, ws_bytes, kStatusBytes + proj_partial_bytes(dims, num_rows))) != DSA_OK)
+    return st;
+  if (num_rows == 0) return DSA_OK;
+  CHECK_ARG(o && w_uv && w_out && u && y, "a tensor pointer is NULL");
+  CHECK_ARG(aligned(o, 16) && aligned(w_uv, 16) && aligned(w_out, 16) && aligned(u, 16) &&
+                aligned(y, 16),
+            "tensors must be 16-byte aligned");
+  if (tensor_map_encoder() == nullptr) {
+    set_error("output projection needs cuTensorMapEncodeTiled from the driver");
+    return DSA_ERR_UNSUPPORTED;
+  }
+  ProjArgs a{};
+  a.num_rows = num_rows;
+  a.n_heads = dims->n_heads;
+  a.d_c = dims->d_c;
+  a.d_v = dims->d_v;
+  a.d_model = dims->d_model;
+  a.o = o;
+  a.w_uv = w_uv;
+  a.w_out = w_out;
+  a.u = u;
+  a.y = y;
+  a.partial = reinterpret_cast<float*>(at(ws, kStatusBytes));
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  return launch_out_proj(a, (cudaStream_t)stream);
 }
 
 }  // extern "C"

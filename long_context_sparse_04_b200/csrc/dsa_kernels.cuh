@@ -97,6 +97,23 @@ size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
 dsa_status launch_cache_append(const AppendArgs& a, cudaStream_t stream);
 int cache_append_max_d_idx();
 
+// Output projection: u = W_UV,i o_i per head, then y = W_out [u_1; ...; u_H].
+struct ProjArgs {
+  int num_rows, n_heads, d_c, d_v, d_model;
+  const void* o;              // [T, H, d_c] bf16
+  const void* w_uv;           // [H, d_v, d_c] bf16
+  const void* w_out;          // [d_model, H * d_v] bf16
+  void* u;                    // [T, H, d_v] bf16
+  void* y;                    // [T, d_model] bf16
+  float* partial;             // workspace: [splits, T, d_model] fp32 (splits > 1)
+  DeviceStatus* status;
+};
+int out_proj_splits(int num_rows, int d_model, int k_blocks);
+dsa_status launch_out_proj(const ProjArgs& a, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled from the driver (null when unavailable), looked up once.
+void* tensor_map_encoder();
+
 // Per-device host state.  Kernel attributes and device properties belong to a
 // device, so a process that drives several GPUs sets and caches them per
 // device (the current one at the call).

@@ -407,15 +407,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
 // 2D byte tensor [rows, 128] with 128-byte rows, box 128 x box_rows, 128B swizzle.
@@ -482,6 +474,17 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+void* tensor_map_encoder() {
+  static void* fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = p;
+  }
+  return fn;
+}
 
 bool indexer_tc_supported(const IndexerArgs& a) {
   if (a.idx_dtype != DSA_FP8_E4M3 || a.d_idx != kDI || a.n_idx_heads != kHI) return false;

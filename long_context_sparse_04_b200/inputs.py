@@ -29,6 +29,7 @@ import numpy as np
 
 # tensor ids of the seed sequences
 TID_QIDX, TID_W, TID_KIDX, TID_LATENT, TID_Q, TID_PLANT, TID_LEN, TID_TABLE = range(1, 9)
+TID_WUV, TID_WOUT, TID_O = 9, 10, 11
 BLOCK = 64          # tokens per page of paged caches
 CHUNK = 1024        # keys per seeded chunk of a sequence (a multiple of BLOCK)
 E4M3_MAX = 448.0
@@ -59,6 +60,8 @@ class DSAConfig:
     std_q: float
     std_kv: float
     seed: int
+    d_v: int = 128          # value head width after W_UV (output projection)
+    d_model: int = 7168     # model width after W_out (output projection)
 
     @property
     def d_qk(self) -> int:
@@ -239,6 +242,30 @@ def new_tokens(cfg: DSAConfig):
     seq = np.repeat(np.arange(cfg.n_seqs, dtype=np.int32), nq)
     j = np.tile(np.arange(nq), cfg.n_seqs)
     return seq, (ctx[seq] - nq + j).astype(np.int32)
+
+
+def out_proj_weights(cfg: DSAConfig):
+    """W_UV [H, d_v, d_c] ~ N(0, 1/d_c) and W_out [d_model, H*d_v] ~ N(0, 1/(H*d_v))
+    (variances), as bf16 bit patterns: unit-scale projections of unit-scale
+    inputs."""
+    w_uv = _normal(cfg.seed, TID_WUV, (0,), (cfg.n_heads, cfg.d_v, cfg.d_c), 1 / math.sqrt(cfg.d_c))
+    w_out = np.empty((cfg.d_model, cfg.n_heads * cfg.d_v), np.float32)
+    step = 512
+    for i in range(0, cfg.d_model, step):
+        r = min(step, cfg.d_model - i)
+        w_out[i:i + r] = _normal(cfg.seed, TID_WOUT, (i // step,), (r, cfg.n_heads * cfg.d_v),
+                                 1 / math.sqrt(cfg.n_heads * cfg.d_v))
+    return to_bf16_bits(w_uv), to_bf16_bits(w_out)
+
+
+def latent_out_rows(cfg: DSAConfig, rows) -> np.ndarray:
+    """Stand-ins for the sparse attention's latent output o [len(rows), H, d_c]
+    (a softmax-weighted mean of unit-variance latent rows, so smaller than
+    one): N(0, 0.1^2), bf16 bit patterns, seeded per row."""
+    if len(rows) == 0:
+        return np.zeros((0, cfg.n_heads, cfg.d_c), np.uint16)
+    return to_bf16_bits(np.stack([_normal(cfg.seed, TID_O, (int(t),), (cfg.n_heads, cfg.d_c), 0.1)
+                                  for t in rows]))
 
 
 def context_lengths(cfg: DSAConfig) -> np.ndarray:
