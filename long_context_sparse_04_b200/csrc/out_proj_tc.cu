@@ -306,7 +306,7 @@ dsa_status launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const GemmA
 int out_proj_splits(int num_rows, int d_model, int k_blocks) {
   const int64_t tiles = (int64_t)((num_rows + kBM - 1) / kBM) * ((d_model + kMaxBN - 1) / kMaxBN);
   const int sms = device_sm_count();
-  if (tiles >= sms) return 1;
+  if (tiles == 0 || tiles >= sms) return 1;
   int s = (int)(sms / tiles);
   s = std::min(s, std::max(1, k_blocks / 8));
   return std::max(1, std::min(s, kMaxSplits));

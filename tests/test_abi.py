@@ -95,6 +95,21 @@ def test_workspace_size_plans():
     assert N.dsa_workspace_size(dims, rows_bad, N.DSA_OP_TOPK) == 0
 
 
+def test_cache_append_and_projection_workspace_sizes():
+    N = _lib()
+    assert N.dsa_workspace_size(_dims(N), None, N.DSA_OP_CACHE_APPEND) == 256
+    p = N.dsa_proj_dims(n_heads=128, d_c=512, d_v=128, d_model=7168)
+    assert N.dsa_output_projection_ws_size(p, 0) == 256          # no rows: status block only
+    # a small batch splits K: status block + fp32 partials [splits, T, d_model]
+    dec = N.dsa_output_projection_ws_size(p, 32)
+    assert dec > 256 and (dec - 256) % (32 * 7168 * 4) == 0 and dec - 256 <= 16 * 32 * 7168 * 4
+    assert N.dsa_output_projection_ws_size(p, 65536) == 256      # enough tiles: no split
+    for bad in (dict(d_c=100), dict(d_v=48), dict(d_v=512), dict(d_model=100), dict(n_heads=0)):
+        kw = dict(n_heads=128, d_c=512, d_v=128, d_model=7168)
+        kw.update(bad)
+        assert N.dsa_output_projection_ws_size(N.dsa_proj_dims(**kw), 8) == 0, bad
+
+
 def test_argument_errors_are_reported_before_any_cuda_call():
     N = _lib()
     fake = ctypes.c_void_p(1 << 20)
