@@ -42,6 +42,10 @@ section and equation on that page):
   module: the output projection after the path, u_{t,i} = W_UV,i o_{t,i} per
   head (W_UV,i is constant in s, so it moves out of the softmax sum) and
   y_t = W_out [u_{t,1}; ...; u_{t,H}].
+* section "Training Mechanics: Dense Warm-Up and KL Alignment", Phase 1: the
+  teacher distribution (dense attention probabilities summed over heads and
+  normalised over the keys), the KL loss of the indexer's softmax against it,
+  and the backward of that loss through the indexer to q_I, w and k_I.
 * section "The Classical Multi-Head Latent Attention (MLA) Mechanism", logit
   equation A_{t,s,i}: the dense MLA that sparse MLA must equal when k covers
   every visible key, and the un-absorbed form used for the absorbed ==
@@ -422,3 +426,59 @@ def output_projection_row(o: np.ndarray, w_uv: np.ndarray, w_out: np.ndarray):
     u = np.einsum("ivc,ic->iv", w_uv, o)
     y = w_out @ u.reshape(-1)
     return u, y
+
+
+# ----------------------------------------------------------------------------
+# Indexer warm-up: KL loss against the dense attention, and its backward
+# ----------------------------------------------------------------------------
+#
+# "DeepSeek Sparse Attention DSA Architecture Guide", section "Training
+# Mechanics: Dense Warm-Up and KL Alignment", "Phase 1: Dense Warm-Up via
+# Teacher-Student Distillation": the teacher distribution of row t is the
+# dense attention probabilities summed over the heads and normalised over the
+# visible keys, p_{t,s} = sum_i A_{t,s,i} / sum_{s'} sum_i A_{t,s',i}, and the
+# indexer minimises L^I = sum_t KL(p_{t,:} || Softmax(I_{t,:})).  Only the
+# indexer's inputs (its queries, keys and head weights) receive gradients.
+
+def dense_attention_probs(q: np.ndarray, kv: np.ndarray, sm_scale: float) -> np.ndarray:
+    """A[i, s] = softmax_s(sm_scale * q[i] . kv[s]) over all given keys (the
+    row's visible keys), q [H, D], kv [n, D].  Returns [H, n]."""
+    z = sm_scale * (q @ kv.T)
+    z = z - z.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def teacher_distribution(a: np.ndarray) -> np.ndarray:
+    """p[s] = sum_i A[i, s] / sum_s' sum_i A[i, s'] for one row, A [H, n]."""
+    tot = a.sum(axis=0)
+    return tot / tot.sum()
+
+
+def indexer_kl_row(p: np.ndarray, scores: np.ndarray):
+    """KL(p || softmax(I)) of one row and its gradient with respect to I.
+
+    KL = sum_s p_s (log p_s - log softmax(I)_s), with 0 log 0 = 0.  Since
+    sum_s p_s = 1, dKL/dI_s = softmax(I)_s - p_s.  Returns (kl, grad [n])."""
+    p = np.asarray(p, dtype=np.float64)
+    scores = np.asarray(scores, dtype=np.float64)
+    m = scores.max()
+    log_z = m + np.log(np.exp(scores - m).sum())
+    log_q = scores - log_z
+    nz = p > 0
+    kl = float(np.sum(p[nz] * (np.log(p[nz]) - log_q[nz])))
+    return kl, np.exp(log_q) - p
+
+
+def indexer_backward_row(q: np.ndarray, w: np.ndarray, k: np.ndarray, g: np.ndarray):
+    """Backward of I[s] = sum_j w[j] ReLU(q[j] . k[s]) for one row, given
+    g[s] = dL/dI[s].  q [H_I, d_I], w [H_I], k [n, d_I], g [n].  ReLU's
+    derivative is 1 where its argument is > 0 and 0 elsewhere (0 at 0).
+    Returns (dq [H_I, d_I], dw [H_I], dk [n, d_I])."""
+    d = k @ q.T                               # [n, H_I]
+    on = (d > 0).astype(np.float64)
+    dw = np.maximum(d, 0.0).T @ g             # [H_I]
+    gd = (g[:, None] * on) * w[None, :]       # dL/d(q_j . k_s), [n, H_I]
+    dq = gd.T @ k                             # [H_I, d_I]
+    dk = gd @ q                               # [n, d_I]
+    return dq, dw, dk

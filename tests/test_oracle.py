@@ -10,6 +10,7 @@ import os
 import numpy as np
 import pytest
 import scipy.special
+import scipy.stats
 
 from oracle import dsa_ref as R
 from long_context_sparse_04_b200 import inputs as I
@@ -467,3 +468,93 @@ def test_output_projection_completes_the_pages_module():
     attn = torch.einsum("is,siv->iv", p, v).reshape(H * d_v)
     y_page = F.linear(attn, t(w_out)).numpy()
     np.testing.assert_allclose(y, y_page, rtol=1e-11, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# P11: indexer warm-up loss (KL to the dense attention) and its backward
+# --------------------------------------------------------------------------
+
+def _warmup_case(seed=22, H=3, D=10, H_I=4, d_I=6, n=9):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((H, D)), rng.standard_normal((n, D)), rng.standard_normal((H_I, d_I)),
+            rng.standard_normal(H_I), rng.standard_normal((n, d_I)))
+
+
+def test_teacher_is_the_head_mean_of_the_dense_attention():
+    # every head's probabilities sum to 1 over the keys, so the normaliser of
+    # the page's teacher is H: p is the mean over heads
+    q, kv, _, _, _ = _warmup_case()
+    a = R.dense_attention_probs(q, kv, 0.3)
+    np.testing.assert_allclose(a.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    p = R.teacher_distribution(a)
+    np.testing.assert_allclose(p, a.mean(axis=0), rtol=1e-14)
+    np.testing.assert_allclose(p.sum(), 1.0, rtol=0, atol=1e-14)
+    # the dense probabilities equal scipy's softmax of the same logits
+    np.testing.assert_allclose(a, scipy.special.softmax(0.3 * q @ kv.T, axis=1), rtol=1e-13)
+
+
+def test_kl_matches_scipy_and_vanishes_at_the_teacher():
+    rng = np.random.default_rng(23)
+    p = rng.random(12)
+    p[3] = 0.0                                   # a key with no teacher mass
+    p /= p.sum()
+    scores = rng.standard_normal(12) * 2
+    kl, _ = R.indexer_kl_row(p, scores)
+    ref = scipy.stats.entropy(p, scipy.special.softmax(scores))
+    assert abs(kl - ref) <= 1e-13 * max(1.0, ref) and kl > 0
+    pp = p + 1e-3
+    pp /= pp.sum()
+    kl0, g0 = R.indexer_kl_row(pp, np.log(pp) + 7.5)      # softmax(log p + c) = p
+    assert abs(kl0) < 1e-14 and np.abs(g0).max() < 1e-14
+
+
+def test_kl_gradient_against_finite_differences_and_autograd():
+    import torch
+    rng = np.random.default_rng(24)
+    p = rng.random(7)
+    p /= p.sum()
+    scores = rng.standard_normal(7)
+    _, g = R.indexer_kl_row(p, scores)
+    h = 1e-6
+    fd = np.array([(R.indexer_kl_row(p, scores + h * e)[0] - R.indexer_kl_row(p, scores - h * e)[0]) / (2 * h)
+                   for e in np.eye(7)])
+    np.testing.assert_allclose(g, fd, rtol=1e-6, atol=1e-9)
+    s = torch.tensor(scores, requires_grad=True)
+    torch.nn.functional.kl_div(torch.log_softmax(s, 0), torch.tensor(p), reduction="sum").backward()
+    np.testing.assert_allclose(g, s.grad.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_indexer_backward_against_autograd():
+    """The warm-up chain for two rows, differentiated by torch autograd: teacher
+    from the dense attention, scores from the indexer definition, KL summed over
+    rows; the oracle's composed gradients must match for q_I, w and k_I."""
+    import torch
+    rng = np.random.default_rng(25)
+    H, D, H_I, d_I, n, T = 3, 10, 4, 6, 9, 2
+    qm = rng.standard_normal((T, H, D))
+    kv = rng.standard_normal((n, D))
+    qi = rng.standard_normal((T, H_I, d_I))
+    w = rng.standard_normal((T, H_I))
+    k = rng.standard_normal((n, d_I))
+    klen = [6, 9]                                 # causal: row t sees its first klen keys
+    dq_o, dw_o, dk_o, loss_o = np.zeros_like(qi), np.zeros_like(w), np.zeros_like(k), 0.0
+    for t in range(T):
+        p = R.teacher_distribution(R.dense_attention_probs(qm[t], kv[:klen[t]], 0.25))
+        sc = R.indexer_row(qi[t], w[t], k[:klen[t]])
+        kl, g = R.indexer_kl_row(p, sc)
+        dq, dw, dk = R.indexer_backward_row(qi[t], w[t], k[:klen[t]], g)
+        dq_o[t], dw_o[t] = dq, dw
+        dk_o[:klen[t]] += dk
+        loss_o += kl
+    tq, tw, tk = (torch.tensor(x, requires_grad=True) for x in (qi, w, k))
+    loss = 0
+    for t in range(T):
+        a = torch.softmax(0.25 * torch.tensor(qm[t]) @ torch.tensor(kv[:klen[t]]).T, dim=1)
+        p = a.sum(0) / a.sum()
+        sc = torch.relu(tk[:klen[t]] @ tq[t].T) @ tw[t]
+        loss = loss + torch.nn.functional.kl_div(torch.log_softmax(sc, 0), p, reduction="sum")
+    loss.backward()
+    assert abs(loss.item() - loss_o) <= 1e-12 * abs(loss_o)
+    np.testing.assert_allclose(dq_o, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dw_o, tw.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk_o, tk.grad.numpy(), rtol=1e-10, atol=1e-12)

@@ -99,6 +99,30 @@ def _bad_outproj_head0_weights(o, w_uv, w_out):
     return u, w_out @ u.reshape(-1)
 
 
+def _bad_kl_grad_sign(p, scores):
+    kl, g = R_orig_kl(p, scores)
+    return kl, -g
+
+
+def _bad_teacher_unnormalised(a):
+    return a.sum(axis=0)
+
+
+def _bad_backward_no_relu_mask(q, w, k, g):
+    d = k @ q.T
+    dw = np.maximum(d, 0.0).T @ g
+    gd = g[:, None] * w[None, :]
+    return gd.T @ k, dw, gd @ q
+
+
+def _bad_backward_dk_without_w(q, w, k, g):
+    dq, dw, _ = R_orig_bwd(q, w, k, g)
+    on = (k @ q.T > 0).astype(np.float64)
+    return dq, dw, (g[:, None] * on) @ q
+
+
+R_orig_kl = R.indexer_kl_row
+R_orig_bwd = R.indexer_backward_row
 R_orig_rows = R.physical_rows
 R_orig_mla = R.sparse_mla_row
 R_orig_e4m3 = R.e4m3_decode
@@ -125,6 +149,13 @@ CASES = [
      [P.test_output_projection_brute_force, P.test_output_projection_completes_the_pages_module]),
     ("output_projection_row", _bad_outproj_head0_weights,
      [P.test_output_projection_brute_force, P.test_output_projection_completes_the_pages_module]),
+    ("indexer_kl_row", _bad_kl_grad_sign,
+     [P.test_kl_gradient_against_finite_differences_and_autograd,
+      P.test_indexer_backward_against_autograd]),
+    ("teacher_distribution", _bad_teacher_unnormalised,
+     [P.test_teacher_is_the_head_mean_of_the_dense_attention, P.test_indexer_backward_against_autograd]),
+    ("indexer_backward_row", _bad_backward_no_relu_mask, [P.test_indexer_backward_against_autograd]),
+    ("indexer_backward_row", _bad_backward_dk_without_w, [P.test_indexer_backward_against_autograd]),
     ("physical_rows", _bad_physical_rows_mirrored_offset,
      [lambda: P.test_cache_append_writes_where_the_layout_says(True)]),
 ]
