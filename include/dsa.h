@@ -336,7 +336,9 @@ size_t dsa_output_projection_ws_size(const dsa_proj_dims* dims, int32_t num_rows
  *   y     [T, d_model] bf16 out
  * All device pointers, 16-byte aligned, owned by the caller; u and y must not
  * overlap the inputs.  ws: dsa_output_projection_ws_size bytes, 256-byte
- * aligned (status block, then split-K partials).  T = 0 launches nothing. */
+ * aligned (status block, then split-K partials); zero its status block once
+ * with dsa_workspace_init.  A bounded wait that runs out is recorded there
+ * (DSA_ERR_TIMEOUT).  T = 0 launches nothing. */
 dsa_status dsa_output_projection(const dsa_proj_dims* dims, int32_t num_rows, const void* o,
                                  const void* w_uv, const void* w_out, void* u, void* y,
                                  void* ws, size_t ws_bytes, dsa_stream_t stream);
