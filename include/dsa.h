@@ -58,7 +58,7 @@ typedef struct CUstream_st* dsa_stream_t;
 typedef enum {
   DSA_OK = 0,
   DSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, bad layout */
-  DSA_ERR_UNSUPPORTED = 2,   /* shape/dtype combination this build does not run   */
+  DSA_ERR_UNSUPPORTED = 2,   /* shape/dtype combination the library does not run */
   DSA_ERR_CUDA = 3,          /* a CUDA call or kernel launch failed               */
   DSA_ERR_OUT_OF_RANGE = 4,  /* device: block-table entry outside [0, num_pages)   */
   DSA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out     */
