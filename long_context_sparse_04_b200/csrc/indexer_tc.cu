@@ -475,14 +475,15 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
 }  // namespace
 
 void* tensor_map_encoder() {
-  static void* fn = nullptr;
-  if (fn == nullptr) {
+  // a function-local static: initialised once, safely under concurrent first calls
+  static void* const fn = [] {
     cudaDriverEntryPointQueryResult q;
     void* p = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess && q == cudaDriverEntryPointSuccess)
-      fn = p;
-  }
+      return p;
+    return static_cast<void*>(nullptr);
+  }();
   return fn;
 }
 
