@@ -126,13 +126,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   const int t = unit / a.splits, sp = unit % a.splits;
   pdl_launch_dependents();
 
-  const int klen = a.row_klen[t];
-  const int nsel = min(klen, a.topk);
-  const int k0 = sp * keys_per_split;
-  const int nvalid = max(0, min(nsel - k0, keys_per_split));
-  const int nblk = (nvalid + kBlk - 1) / kBlk;
-  const int seq = a.row_seq[t];
-
+  // Setup that reads no input memory overlaps the predecessor's tail: barrier
+  // init and the TMEM allocation.  Every read of an input (row lengths, Q, the
+  // selection, the caches) comes after pdl_wait(), so a predecessor that
+  // writes any of them (and triggers its dependents early) is complete and
+  // visible first.
   if (threadIdx.x == 0) {
     mbar_init(&S.q_full, 128);
     mbar_init(&S.x_full, 1);                 // armed by this CTA, completed by the peer's copy
@@ -145,15 +143,23 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       mbar_init(&S.pv_done[i], 1);
     }
     fence_mbar_init();
-    if (nblk > 0) mbar_expect_tx(&S.x_full, kXBytes);   // arm the first transfer
   }
   __syncwarp();
   if (warp == 12) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // Q first: it does not depend on the selection (the gather warps arrive on
-  // q_full for these pieces once the barrier init is visible, below)
+  pdl_wait();
+  trace_kernel(a.status, DSA_KERNEL_MLA_TC);
+  const int klen = a.row_klen[t];
+  const int nsel = min(klen, a.topk);
+  const int k0 = sp * keys_per_split;
+  const int nvalid = max(0, min(nsel - k0, keys_per_split));
+  const int nblk = (nvalid + kBlk - 1) / kBlk;
+  const int seq = a.row_seq[t];
+  if (threadIdx.x == 0 && nblk > 0) mbar_expect_tx(&S.x_full, kXBytes);   // arm the first transfer
+  // Q first: its pieces land while the selection is resolved below (the
+  // gather warps arrive on q_full for them once the barrier init is visible)
   if (warp < 4 && nblk > 0) {
     const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
     for (int i = 0; i < kPieces; ++i) {
@@ -166,10 +172,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       }
     }
   }
-  // The selection comes from the previous kernel: everything above (barriers,
-  // TMEM, the Q load) overlaps its tail.
-  pdl_wait();
-  trace_kernel(a.status, DSA_KERNEL_MLA_TC);
   // physical rows of the selected keys of this split (entries past nvalid are
   // none): all index loads of a thread first, then all its block-table loads
   {
