@@ -187,6 +187,21 @@ dsa_status dsa_set_stage_events(void* const* events, int32_t n_events);
  * dev_buf = NULL turns it off.  For performance analysis only. */
 dsa_status dsa_set_trace_buffer(void* dev_buf, size_t bytes);
 
+/* Fault injection, for tests of the failure paths only (never set it in
+ * production).  Every wait inside the kernels is bounded: after a number of
+ * polls it records DSA_ERR_TIMEOUT (detail = the wait's site) in the device
+ * status word and the kernel winds down and returns, with every asynchronous
+ * copy and tensor-core operation it started complete.  On the calling host
+ * thread, later launches use `spin_limit` polls per wait (0 = the built-in
+ * limit) and inject the faults in `faults`:
+ *   DSA_FAULT_INDEXER_ACC_RELEASE  the tensor-core indexer's epilogue never
+ *       releases its accumulators, so its MMA issuer's wait for a free
+ *       accumulator runs out (and then the epilogue's and the producer's
+ *       waits for tiles that are never computed).
+ * Returns DSA_ERR_INVALID_ARG for unknown fault bits.  (0, 0) switches it off. */
+#define DSA_FAULT_INDEXER_ACC_RELEASE 0x1u
+dsa_status dsa_set_fault_injection(uint32_t spin_limit, uint32_t faults);
+
 /* Stage 1: indexer scores.
  *   q_idx   [T, H_I, d_I] e4m3 | f32
  *   q_scale [T, H_I] fp32 (e4m3 only, else NULL): dequantised q = e4m3 * scale
@@ -296,6 +311,13 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
  * with detail n; a token whose key holds an infinity or NaN is not written
  * either, and is recorded as DSA_ERR_INVALID_ARG with detail n (the first
  * error of a launch wins).  The other tokens are written.
+ * Contiguous layout: the library knows where each sequence's rows start
+ * (seq_start) but not where they end, so the only range check is
+ * [0, num_tokens).  A position past the end of sequence b's own rows is
+ * written into the rows that follow them (the next sequence's, in the usual
+ * layout) without an error: the caller keeps tok_pos[n] below the capacity of
+ * its sequence.  The paged layout has no such hazard (a position beyond the
+ * block table's width is refused).
  * ws: at least dsa_workspace_size(dims, NULL, DSA_OP_CACHE_APPEND) bytes (the
  * status block), zeroed once by dsa_workspace_init.  n_new = 0 launches
  * nothing. */

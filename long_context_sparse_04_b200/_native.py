@@ -20,6 +20,7 @@ DSA_KERNEL_INDEXER_SIMT, DSA_KERNEL_INDEXER_TC, DSA_KERNEL_TOPK = 0x01, 0x02, 0x
 DSA_KERNEL_MLA_SIMT, DSA_KERNEL_MLA_TC, DSA_KERNEL_MLA_COMBINE = 0x08, 0x10, 0x20
 DSA_KERNEL_CACHE_APPEND = 0x40
 DSA_KERNEL_OUT_PROJ, DSA_KERNEL_OUT_PROJ_REDUCE = 0x80, 0x100
+DSA_FAULT_INDEXER_ACC_RELEASE = 0x1
 
 
 class dsa_dims(ctypes.Structure):
@@ -59,6 +60,7 @@ _SIGS = {
     "dsa_read_kernel_trace": (ctypes.c_int, [_P, _P, _P]),
     "dsa_set_stage_events": (ctypes.c_int, [_P, ctypes.c_int32]),
     "dsa_set_trace_buffer": (ctypes.c_int, [_P, ctypes.c_size_t]),
+    "dsa_set_fault_injection": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint32]),
     "dsa_indexer_scores": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
                                           ctypes.c_size_t, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P]),
@@ -136,6 +138,11 @@ def dsa_set_stage_events(events):
 
 def dsa_set_trace_buffer(buf, nbytes):
     return _call("dsa_set_trace_buffer", buf, nbytes)
+
+
+def dsa_set_fault_injection(spin_limit: int, faults: int, check=True):
+    """Tests only: bounded-wait poll limit and DSA_FAULT_* bits of this thread's launches."""
+    return _call("dsa_set_fault_injection", spin_limit, faults, check=check)
 
 
 def dsa_indexer_scores(dims, rows, cache, q_idx, q_scale, w, scores, ld_scores, ws, ws_bytes,

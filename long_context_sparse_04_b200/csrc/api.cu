@@ -15,12 +15,15 @@ static thread_local cudaEvent_t g_stage_ev[4] = {nullptr, nullptr, nullptr, null
 static thread_local int g_n_stage_ev = 0;
 
 static thread_local long long* g_trace = nullptr;
+static thread_local uint32_t g_fault_spin = 0, g_fault_inject = 0;
 
 static void stage_event(int i, cudaStream_t s) {
   if (g_n_stage_ev == 4 && g_stage_ev[i] != nullptr) cudaEventRecord(g_stage_ev[i], s);
 }
 
 long long* trace_buffer() { return g_trace; }
+uint32_t fault_spin_limit() { return g_fault_spin ? g_fault_spin : kSpinLimit; }
+uint32_t fault_inject() { return g_fault_inject; }
 
 dsa_status set_smem_limit_once(const void* fn, size_t bytes, std::atomic<bool> (&done)[kMaxDevices]) {
   int dev = 0;
@@ -414,6 +417,16 @@ dsa_status dsa_set_trace_buffer(void* dev_buf, size_t bytes) {
     return DSA_ERR_INVALID_ARG;
   }
   g_trace = static_cast<long long*>(dev_buf);
+  return DSA_OK;
+}
+
+dsa_status dsa_set_fault_injection(uint32_t spin_limit, uint32_t faults) {
+  if ((faults & ~(uint32_t)DSA_FAULT_INDEXER_ACC_RELEASE) != 0) {
+    set_error("unknown fault bits 0x%x", faults);
+    return DSA_ERR_INVALID_ARG;
+  }
+  g_fault_spin = spin_limit;
+  g_fault_inject = faults;
   return DSA_OK;
 }
 

@@ -96,8 +96,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 // Bounded wait; on time-out records DSA_ERR_TIMEOUT (detail = site) and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DeviceStatus* st,
-                                          int site) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+                                          int site, uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   set_status(st, DSA_ERR_TIMEOUT, site);
   return false;
@@ -180,6 +180,11 @@ __device__ __forceinline__ void cp_async_16_zfill(void* smem_dst, const void* gm
 __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
                : "memory");
+}
+// 4-byte copy that reads nothing and writes zeros when `valid` is false.
+__device__ __forceinline__ void cp_async_4_zfill(void* smem_dst, const void* gmem_src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src), "r"(valid ? 4 : 0) : "memory");
 }
 // Arrive on `bar` once all cp.async issued so far by this thread have landed
 // (the arrival counts toward the barrier's expected count).

@@ -77,6 +77,11 @@ struct AppendArgs {
 
 // Profiling trace buffer registered on the calling host thread (or null).
 long long* trace_buffer();
+// Test-only fault injection of the calling host thread (dsa_set_fault_injection):
+// the spin limit of the kernels' bounded waits (kSpinLimit unless set) and the
+// DSA_FAULT_* bits to inject.
+uint32_t fault_spin_limit();
+uint32_t fault_inject();
 static constexpr int kTraceEvents = 8, kTraceBlocks = 32;
 
 dsa_status launch_indexer_simt(const IndexerArgs& a, cudaStream_t stream);

@@ -16,11 +16,13 @@
 // physical cache row of both 64-key halves of every tile of the range into
 // shared memory, so the loops below never wait on a dependent global load.
 // Roles (576 threads):
-//   warp 0      producer (one thread): TMA of the two 64-row key boxes (a box
-//               never crosses a 64-token page) into a 10-stage ring (6 when
-//               N = 256), and of the group's queries (N x 128 B) into a double
-//               buffer.  Per-tile flags computed in the prologue (first / last
-//               tile of its group) keep this loop short.
+//   warp 0      producer: one thread issues the TMA of the two 64-row key
+//               boxes (a box never crosses a 64-token page) into a 10-stage
+//               ring (6 when N = 256), and of the group's queries (N x 128 B)
+//               into a double buffer; the 32 lanes copy the tile's 128 key
+//               scales into a scale slot with cp.async, so the epilogue never
+//               waits on a global load.  Per-tile flags computed in the
+//               prologue (first / last tile of its group) keep this loop short.
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
 //               into one of four (N <= 128) or two TMEM accumulators; one
@@ -47,6 +49,13 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 2048;
 constexpr int kMaxCtaTiles = 512;
 constexpr int kKeyTileBytes = kTileKeys * kDI;   // 16 KB
+// Key-scale slots: the producer writes tile j's scales into slot j % 16 when it
+// fills the tile's key stage, and the epilogue reads them before it releases
+// the tile's accumulator.  The producer reaches tile j + 16 only after the MMA
+// of tile j + 16 - stages, which needs the accumulator of tile
+// j + 16 - stages - accumulators >= j released: 16 >= stages + accumulators
+// (10 + 4, or 6 + 2) keeps a slot from being overwritten before it is read.
+constexpr int kScaleSlots = 16;
 
 // Key-tile stages in flight: as many as shared memory allows beside the queries.
 template <int NQ>
@@ -61,6 +70,7 @@ struct __align__(1024) IdxSmem {
   uint8_t keys[num_stages<NQ>()][kKeyTileBytes];
   uint8_t q[2][NQ * kHI * kDI];
   float wq[kEpiWarps][kHI];                             // per epilogue warp: w' of its heads
+  float kscale[kScaleSlots][kTileKeys];                 // key scales of tile j in slot j % kScaleSlots
   int32_t tile_row[kMaxCtaTiles][2];                    // physical row of each 64-key half, -1: none
   int32_t tile_info[kMaxCtaTiles];                      // group << 2 | last tile of group << 1 | first
   int32_t tile_off[kMaxGroups + 1];
@@ -73,6 +83,8 @@ struct __align__(1024) IdxSmem {
 
 struct TcArgs {
   long long* trace;           // profiling stamps (CTA 0, first 32 tiles) or null
+  uint32_t spin_limit;        // polls of every bounded wait
+  uint32_t inject;            // DSA_FAULT_* bits (tests only)
   int num_rows, n_groups;
   const int32_t* row_seq;
   const int32_t* row_klen;
@@ -152,6 +164,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   IdxSmem<NQ>& S = *reinterpret_cast<IdxSmem<NQ>*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t lim = a.spin_limit;
   pdl_launch_dependents();
   pdl_wait();
   trace_kernel(a.status, DSA_KERNEL_INDEXER_TC);
@@ -189,7 +202,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (threadIdx.x == 0) S.tile_off[0] = 0;
   }
   if (threadIdx.x == 32) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], 1); }
+    // full: the producer lane's arrive (with the key bytes as transactions)
+    // plus one cp.async arrival per producer lane for the scales
+    for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 33); mbar_init(&S.empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
@@ -240,13 +255,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   const bool run = ntile > 0 && ntile <= kMaxCtaTiles;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer (lane 0): TMA only
-    if (run && lane == 0) {
-      // A lean loop: one thread issues every load, so its instruction count
-      // per tile bounds the tile rate.
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_q);
-      const bool tracing = a.trace != nullptr && blockIdx.x == 0;
+    // ------------------------------------------------------------ producer
+    // Lane 0 issues the TMA loads of the keys (and of the queries); every lane
+    // then copies 4 of the tile's 128 key scales into the scale slot with
+    // cp.async, whose completion also arrives on the stage's full barrier.
+    if (run) {
+      // A lean loop: one thread issues every bulk load, so its instruction
+      // count per tile bounds the tile rate.
+      if (lane == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_q);
+      }
+      const bool tracing = a.trace != nullptr && blockIdx.x == 0 && lane == 0;
+      const int half = lane >> 4, k4 = 4 * (lane & 15);
       int st = 0, qb = 0;
       uint32_t ph = 1, qph = 1;                       // parity to wait for on empty / q_empty
       int qcount = 0, j = 0;
@@ -254,36 +275,75 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       for (; j < ntile; ++j) {
         const int info = S.tile_info[j];
         const int2 rr = *reinterpret_cast<const int2*>(S.tile_row[j]);
-        if (info & 1) {
-          if (qcount > 0) { qb ^= 1; if (qb == 0) qph ^= 1; }
-          ++qcount;
-          if (!(alive = mbar_wait(&S.q_empty[qb], qph, a.status, 1))) break;
-          mbar_expect_tx(&S.q_full[qb], kQBytes);
-          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, (info >> 2) * NQ * kHI);
+        if (lane == 0) {
+          if (info & 1) {
+            if (qcount > 0) { qb ^= 1; if (qb == 0) qph ^= 1; }
+            ++qcount;
+            alive = mbar_wait(&S.q_empty[qb], qph, a.status, 1, lim);
+            if (alive) {
+              mbar_expect_tx(&S.q_full[qb], kQBytes);
+              tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, (info >> 2) * NQ * kHI);
+            }
+          }
+          alive = alive && mbar_wait(&S.empty[st], ph, a.status, 2, lim);
         }
-        if (!(alive = mbar_wait(&S.empty[st], ph, a.status, 2))) break;
-        if (tracing) istamp(a.trace, 0, j);
-        const uint32_t bytes = (rr.x >= 0 ? kKeyTileBytes / 2 : 0) + (rr.y >= 0 ? kKeyTileBytes / 2 : 0);
-        if (bytes == 0) {
-          mbar_arrive(&S.full[st]);
-        } else {
-          mbar_expect_tx(&S.full[st], bytes);
-          if (rr.x >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, rr.x);
-          if (rr.y >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, rr.y);
+        alive = __shfl_sync(0xffffffffu, alive, 0);   // uniform: the stage is free
+        if (!alive) break;
+        if (lane == 0) {
+          if (tracing) istamp(a.trace, 0, j);
+          const uint32_t bytes = (rr.x >= 0 ? kKeyTileBytes / 2 : 0) + (rr.y >= 0 ? kKeyTileBytes / 2 : 0);
+          if (bytes == 0) {
+            mbar_arrive(&S.full[st]);
+          } else {
+            mbar_expect_tx(&S.full[st], bytes);
+            if (rr.x >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, rr.x);
+            if (rr.y >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, rr.y);
+          }
+          if (tracing) istamp(a.trace, 1, j);
         }
-        if (tracing) istamp(a.trace, 1, j);
+        // scales of keys [64 half + k4, +4): one 16-byte piece when aligned and in
+        // range, else four 4-byte pieces (rows past the cache read as 0)
+        {
+          const int row = half ? rr.y : rr.x;
+          float* dst = &S.kscale[j % kScaleSlots][64 * half + k4];
+          const int64_t pr = (int64_t)row + k4;
+          if (row >= 0 && (reinterpret_cast<uintptr_t>(a.k_scale + pr) & 15) == 0 &&
+              pr + 4 <= a.map.num_tokens) {
+            cp_async_16(dst, a.k_scale + pr);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const bool ok = row >= 0 && pr + e < a.map.num_tokens;
+              cp_async_4_zfill(dst + e, a.k_scale + (ok ? pr + e : 0), ok);
+            }
+          }
+          cp_async_mbar_arrive(&S.full[st]);
+        }
         if (++st == kStages) { st = 0; ph ^= 1; }
       }
-      // tail: wait until the MMAs have released every stage and query buffer in
-      // use, so no commit is still in flight to this CTA's shared memory at exit
-      if (alive) {
+      cp_async_wait_all();
+      // tail: every bulk load issued has landed (also when a wait above ran
+      // out and the MMA stopped consuming), then the MMAs have released every
+      // stage and query buffer in use, so nothing is still in flight to this
+      // CTA's shared memory at exit
+      if (lane == 0) {
+        for (int s2 = 0; s2 < kStages && s2 < j; ++s2) {
+          const int fills = (j - 1 - s2) / kStages + 1;
+          if (!mbar_wait(&S.full[s2], (fills - 1) & 1, a.status, 9, lim)) break;
+        }
+        for (int q2 = 0; q2 < 2 && q2 < qcount; ++q2) {
+          const int fills = (qcount - q2 + 1) / 2;
+          if (!mbar_wait(&S.q_full[q2], (fills - 1) & 1, a.status, 10, lim)) break;
+        }
+      }
+      if (alive && lane == 0) {
         for (int s2 = 0; s2 < kStages && s2 < j; ++s2) {
           const int last_use = (j - 1 - s2) / kStages;
-          if (!mbar_wait(&S.empty[s2], last_use & 1, a.status, 7)) break;
+          if (!mbar_wait(&S.empty[s2], last_use & 1, a.status, 7, lim)) break;
         }
         for (int q2 = 0; q2 < 2 && q2 < qcount; ++q2) {
           const int last_use = (qcount - 1 - q2) >> 1;
-          if (!mbar_wait(&S.q_empty[q2], last_use & 1, a.status, 8)) break;
+          if (!mbar_wait(&S.q_empty[q2], last_use & 1, a.status, 8, lim)) break;
         }
       }
     }
@@ -304,11 +364,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         if (info & 1) {
           qb ^= 1;
           if (qb == 0) qph ^= 1;
-          if (!mbar_wait(&S.q_full[qb], qph, a.status, 3)) break;
+          if (!mbar_wait(&S.q_full[qb], qph, a.status, 3, lim)) break;
         }
-        if (!mbar_wait(&S.full[st], ph, a.status, 4)) break;
+        if (!mbar_wait(&S.full[st], ph, a.status, 4, lim)) break;
         if (tracing) istamp(a.trace, 5, j);
-        if (!mbar_wait(&S.acc_empty[ab], aph, a.status, 5)) break;
+        if (!mbar_wait(&S.acc_empty[ab], aph, a.status, 5, lim)) break;
         tc_fence_after();
         if (tracing) istamp(a.trace, 2, j);
         const uint64_t kd = kd0 + (uint64_t)st * kStageStep, qd = qd0 + (uint64_t)qb * kQStep;
@@ -353,17 +413,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           S.wq[e][q] = r < a.num_rows ? a.w[(int64_t)r * kHI + q] * a.q_scale[(int64_t)r * kHI + q] : 0.f;
         __syncwarp();
       }
-      // key scale of this thread's key, loaded before the accumulator wait
-      float ks = 0.f;
-      {
-        const int rr = S.tile_row[j][row_in_tile >> 6];
-        const int64_t pr = (int64_t)rr + (row_in_tile & 63);
-        if (rr >= 0 && pr < a.map.num_tokens) ks = __ldg(a.k_scale + pr);
-      }
       const int ab = j % kAcc;
-      // the stage's barrier completes when the tile's MMAs are done
-      dead = dead || !mbar_wait(&S.empty[j % kStages], (j / kStages) & 1, a.status, 6);
+      // the stage's barrier completes when the tile's MMAs are done, which
+      // also orders the key scales the producer copied for this tile
+      dead = dead || !mbar_wait(&S.empty[j % kStages], (j / kStages) & 1, a.status, 6, lim);
       tc_fence_after();
+      const float ks = S.kscale[j % kScaleSlots][row_in_tile];
       if (threadIdx.x == 64) istamp(a.trace, 4, j);
       const uint32_t col = tmem + lane_off + ab * N + qi * kHI;
       uint32_t v0[32], v1[32];
@@ -373,7 +428,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tmem_wait_ld_regs(v1);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.acc_empty[ab]);      // values are in registers
+      // values are in registers (a test may withhold the release, so that the
+      // MMA issuer's bounded wait runs out)
+      if (lane == 0 && !(a.inject & DSA_FAULT_INDEXER_ACC_RELEASE)) mbar_arrive(&S.acc_empty[ab]);
       // sum_h w'_h ReLU(x_h), two heads per packed fp32x2 FMA
       const ulonglong2* wv = reinterpret_cast<const ulonglong2*>(&S.wq[e][0]);
       unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -452,6 +509,8 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     t.ld = a.ld_scores;
     t.status = a.status;
     t.trace = trace_buffer();
+    t.spin_limit = fault_spin_limit();
+    t.inject = fault_inject();
     CUtensorMap tq;
     if (!make_tmap_rows128(&tq, static_cast<const uint8_t*>(a.q_idx) + (int64_t)r0 * kHI * kDI,
                            (uint64_t)t.num_rows * kHI, NQ * kHI)) {

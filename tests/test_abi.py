@@ -141,3 +141,10 @@ def test_argument_errors_are_reported_before_any_cuda_call():
     assert st == N.DSA_ERR_INVALID_ARG          # num_tokens not a whole number of pages
     with pytest.raises(N.DSAError):
         N.dsa_topk(_dims(N, topk=0), rows, fake, 128, fake, fake, 4096, None)
+
+
+def test_fault_injection_rejects_unknown_bits():
+    # host-side argument check only: no device work
+    N = _lib()
+    assert N.dsa_set_fault_injection(0, 0x80, check=False) == N.DSA_ERR_INVALID_ARG
+    assert N.dsa_set_fault_injection(0, 0) == N.DSA_OK
