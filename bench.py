@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4, help="oracle rows per CPU-baseline sample")
     ap.add_argument("--n-seqs", type=int, default=None, help="smaller batch (profiling captures)")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the 64K prefill measurement that the default decode run adds")
     return ap.parse_args()
 
 
@@ -90,6 +92,13 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
 def throughput(world: int, rows_per_rank: int, steps: int, total_ms: float) -> float:
     """Whole-job query-tokens/s: all ranks' rows over the slowest rank's time."""
     return world * rows_per_rank * steps / (total_ms / 1e3)
+
+
+def path_config(cfg, rows_per_gpu: int, world: int) -> dict:
+    """The `config` object of a path line; both arms print the same one."""
+    return {"workload": workload_desc(cfg), "rows_per_gpu": int(rows_per_gpu),
+            "l2": "flushed before every step (256 MiB write, untimed)",
+            "parallelism": f"{world} independent ranks (weak scaling)"}
 
 
 def workload_desc(cfg) -> str:
@@ -223,7 +232,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": workload_desc(cfg)},
+        "data": "synthetic", "config": path_config(cfg, len(inp["row_seq"]), world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{len(rows)} of {len(inp['row_seq'])} query rows per step "
                                    f"(all three stages, float64 NumPy)"},
@@ -256,29 +265,19 @@ def algorithmic(cfg, inp, stage):
     return {"bytes": by, "flops": fl}
 
 
-def run_ours(args):
-    import numpy as np
+def measure_path(args, cfg, dev, rank: int, world: int, steps: int, warmup: int,
+                 want_e2e: bool, want_cpu: bool) -> dict:
+    """Time `steps` passes of the whole path over one batch of `cfg` on `dev`:
+    device time per step (max over ranks), per-stage breakdown, roofline of the
+    dominant stage, and optionally the end-to-end and host-oracle figures."""
     import torch
-    rank, world, local = dist_info()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
 
-    from long_context_sparse_04_b200 import build
-    build.build()
     from long_context_sparse_04_b200 import _native as N
     from long_context_sparse_04_b200 import inputs as I
     from long_context_sparse_04_b200.workload import DeviceWorkload
 
-    cfg = I.CONFIGS[args.workload]
-    if args.n_seqs:
-        cfg = cfg.replace(n_seqs=args.n_seqs)
     cfg_r = rank_config(cfg, rank)
-    inp = I.generate(cfg_r)
+    inp = I.generate(cfg_r, threads=max(4, min(32, len(os.sched_getaffinity(0)))))
     wl = DeviceWorkload(inp, device=dev)
     T = wl.T
     stream = torch.cuda.current_stream(dev)
@@ -308,7 +307,7 @@ def run_ours(args):
         if world > 1:
             torch.distributed.barrier()
 
-    for _ in range(max(args.warmup, 0)):
+    for _ in range(max(warmup, 0)):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
@@ -331,7 +330,7 @@ def run_ours(args):
     # timed steps: one event pair around each call (events between the
     # kernels of a call would cut their programmatic overlap)
     step_ms = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.zero_()
         step_ev[0].record(stream)
         step()
@@ -347,7 +346,7 @@ def run_ours(args):
         # the three stage calls over the whole batch (the forward runs them
         # per 512-row chunk)
         scores = torch.empty((T, wl.ld), dtype=torch.float32, device=dev)
-        for _ in range(args.steps):
+        for _ in range(steps):
             flush.zero_()
             ev[0].record(stream)
             wl.indexer(scores)
@@ -364,7 +363,7 @@ def run_ours(args):
     else:
         # the library records events between its launches
         N.dsa_set_stage_events([e.cuda_event for e in ev])
-        for _ in range(args.steps):
+        for _ in range(steps):
             flush.zero_()
             wl.decode_step(out=out, lse=lse)
             torch.cuda.synchronize(dev)
@@ -373,16 +372,13 @@ def run_ours(args):
             stage_ms["mla"].append(ev[2].elapsed_time(ev[3]))
         N.dsa_set_stage_events([])
     total_ms = max_over_ranks(sum(step_ms), world, dev)
-    ms_per_step = total_ms / args.steps
-    value = throughput(world, T, args.steps, total_ms)
-    if prefill:   # three kernels per 512-row chunk, no split combine
-        launches_per_step = 3 * ((T + 511) // 512)
-    else:
-        launches_per_step = 3 + (1 if ran & N.DSA_KERNEL_MLA_COMBINE else 0)
+    ms_per_step = total_ms / steps
+    value = throughput(world, T, steps, total_ms)
+    launches_per_step = path_launches(N, ran, T, prefill)
 
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if want_e2e:
         host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("q_idx", "q_scale", "w", "q", "row_klen")
                    if getattr(wl, k) is not None}
         host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -391,7 +387,7 @@ def run_ours(args):
         d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         tot = 0.0
-        for i in range(args.warmup + args.steps):
+        for i in range(warmup + steps):
             flush.zero_()
             e0.record(stream)
             for k, v in host_in.items():
@@ -401,10 +397,10 @@ def run_ours(args):
             host_lse.copy_(lse, non_blocking=True)
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            if i >= args.warmup:
+            if i >= warmup:
                 tot += e0.elapsed_time(e1)
         tot = max_over_ranks(tot, world, dev)
-        e2e = {"value": throughput(world, T, args.steps, tot), "unit": UNIT,
+        e2e = {"value": throughput(world, T, steps, tot), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     # ---- roofline of the dominant kernel
@@ -445,7 +441,7 @@ def run_ours(args):
              "mla": "mla_tc_kernel" if mla_tc else "mla_simt_kernel"}[dom]
     roof = {"kernel": kname, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak if peak else None, "peak_source": peak_kind,
-            "traffic": kernel_traffic(kname, args.workload, alg["bytes"]),
+            "traffic": kernel_traffic(kname, cfg.name, alg["bytes"]),
             "algorithmic_per_launch": alg["bytes"] if bound == "hbm" else alg["flops"]}
     stages = {}
     for k in avg:
@@ -455,7 +451,7 @@ def run_ours(args):
                      "tflops": a["flops"] / s / 1e12}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if want_cpu and rank == 0 and world == 1:
         # bounded sample: about 10-20 s of oracle work on the host cores
         _, t1 = oracle_rows_per_s(inp, sample_rows(inp, 1))
         n = int(max(1, min(T, 12.0 / max(t1, 1e-3))))
@@ -465,19 +461,68 @@ def run_ours(args):
         cpu = {"value": v, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
                "sample": f"{len(rows)} of {T} query rows of one batch x {reps}, all three "
                          f"stages, float64 NumPy, {dt:.1f} s"}
+    del wl, inp, out, lse, idx_out, flush
+    torch.cuda.empty_cache()
+    return {"T": T, "value": value, "ms_per_step": ms_per_step, "steps": steps, "warmup": warmup,
+            "stages": stages, "roofline": roof, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": launches_per_step * steps, "clocks": clk}
+
+
+def path_launches(N, ran: int, T: int, prefill: bool) -> int:
+    """Kernels of this library one step launches."""
+    if prefill:   # three kernels per 512-row chunk, no split combine
+        return 3 * ((T + 511) // 512)
+    return 3 + (1 if ran & N.DSA_KERNEL_MLA_COMBINE else 0)
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from long_context_sparse_04_b200 import build
+    build.build()
+    from long_context_sparse_04_b200 import inputs as I
+
+    cfg = I.CONFIGS[args.workload]
+    if args.n_seqs:
+        cfg = cfg.replace(n_seqs=args.n_seqs)
+    m = measure_path(args, cfg, dev, rank, world, args.steps, args.warmup,
+                     want_e2e=not args.no_e2e, want_cpu=not args.no_cpu_baseline)
+    # The metric names both halves: the 128K decode step is the headline value
+    # and the 64K causal prefill is measured in the same run (one GPU only: a
+    # 64K workload holds ~11 GB of inputs per rank), a few steps of one
+    # dsa_forward over all 65,536 rows each.
+    pre = None
+    if (world == 1 and args.workload == "decode_128k_paged" and not args.n_seqs
+            and not args.no_prefill):
+        p = measure_path(args, I.CONFIGS["prefill_64k"], dev, rank, world, 3, 3,
+                         want_e2e=False, want_cpu=False)
+        pre = {"workload": workload_desc(I.CONFIGS["prefill_64k"]), "value": p["value"],
+               "unit": UNIT, "ms_per_step": p["ms_per_step"], "steps": p["steps"],
+               "warmup": p["warmup"], "stages": p["stages"], "roofline": p["roofline"],
+               "gpu_launches": p["gpu_launches"], "clocks": p["clocks"]}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "metric": METRIC, "value": m["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)",
             "data": "synthetic",
-            "config": {"workload": workload_desc(cfg), "rows_per_gpu": T,
-                       "l2": "flushed before every step (256 MiB write, untimed)",
-                       "parallelism": f"{world} independent ranks (weak scaling)"},
-            "stages": stages, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+            "config": path_config(cfg, m["T"], world),
+            "stages": m["stages"], "roofline": m["roofline"], "cpu_baseline": m["cpu_baseline"],
+            "e2e": m["e2e"],
+            "gpu_launches": m["gpu_launches"],
+            "clocks": m["clocks"],
         }
+        if pre is not None:
+            line["prefill_64k"] = pre
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -363,11 +363,17 @@ def generate(cfg: DSAConfig, with_q: bool = True, threads: int = 8, rows=None) -
     with ThreadPoolExecutor(max_workers=threads) as ex:
         list(ex.map(fill, jobs))
 
-    qf = qidx_rows_f32(cfg, qrows)
-    if cfg.fp8:
-        q_idx, q_scale = to_e4m3_rows(qf)
-    else:
-        q_idx, q_scale = qf, None
+    # indexer queries, in row chunks on the thread pool (every row is seeded on
+    # its own and quantised on its own, so the chunking changes no byte)
+    def qidx_chunk(r):
+        qf = qidx_rows_f32(cfg, r)
+        return to_e4m3_rows(qf) if cfg.fp8 else (qf, None)
+
+    chunks = [qrows[i: i + 1024] for i in range(0, T, 1024)] or [qrows]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        parts = list(ex.map(qidx_chunk, chunks))
+    q_idx = np.concatenate([p[0] for p in parts])
+    q_scale = np.concatenate([p[1] for p in parts]) if cfg.fp8 else None
     w = w_rows(cfg, qrows)
     inp = dict(row_seq=row_seq, row_klen=row_klen, q_idx=q_idx, q_scale=q_scale, w=w,
                k_idx=k_idx, k_scale=k_scale, latent=latent, cache=cache,

@@ -82,7 +82,10 @@ def _compare(got, want):
 
 def _scattered_tokens(inp, cfg, n, rng):
     """n distinct (seq, pos) pairs inside the sequences' pages, the last
-    position of every sequence among them."""
+    position of every sequence among them.  Each position stays inside its own
+    sequence's rows: the generator gives every sequence a page-rounded region
+    (contiguous layout: seq_start[b] is a multiple of 64 and the region holds
+    ceil(ctx/64)*64 rows), and positions are drawn below that size."""
     ctx = I.context_lengths(cfg)
     pages = -(-ctx // I.BLOCK) * I.BLOCK
     pairs = {(b, int(ctx[b]) - 1) for b in range(len(ctx))}

@@ -3,11 +3,12 @@
 The decode workloads run whole through dsa_decode_step, the call bench.py
 times, with the scores and indices also written out; every row is checked for
 the properties that hold at any size and a sample of rows against the oracle.
-The 8K prefill runs whole through dsa_forward (512-row chunks); the scores of
-its sampled rows come from a second, stage-by-stage run on those rows alone
-(per-row results do not depend on the batch, which the test also checks). The
-64K prefill runs its sampled query rows alone against the full 64K-token
-caches: full key length, full top-k width, full gather range per row.
+The 8K and 64K prefills run whole through dsa_forward (512-row chunks), the
+call bench.py times; the scores of their sampled rows come from a second,
+stage-by-stage run on those rows alone (per-row results do not depend on the
+batch, which the tests also check).  The 64K outputs are too large to copy out,
+so their every-row properties are checked on the device.  The 64K prefill also
+runs its sampled query rows alone against the full 64K-token caches.
 """
 import numpy as np
 import pytest
@@ -88,6 +89,56 @@ def test_prefill_8k_full(N):
     s_sc, s_idx = P.to_np(s_sc), P.to_np(s_idx)
     assert np.array_equal(s_idx, idx[sample]), "selection depends on the batch"
     P.check_rows(sub, range(len(sample)), s_sc, idx[sample], out[sample], lse[sample])
+
+
+def _check_selection_properties_device(row_klen, k, idx, out, lse):
+    """_check_selection_properties for workloads too large to copy out: the
+    same checks on every row, as tensor reductions on the device."""
+    import torch
+    T = idx.shape[0]
+    klen = torch.as_tensor(np.asarray(row_klen, dtype=np.int64), device=idx.device).view(T, 1)
+    col = torch.arange(k, device=idx.device, dtype=torch.int64).view(1, k)
+    kk = torch.clamp(klen, max=k)
+    sel = col < kk
+    ix = idx.to(torch.int64)
+    assert bool(((ix >= 0) & (ix < klen))[sel].all()), "index out of range"
+    asc = ix[:, 1:] > ix[:, :-1]
+    assert bool(asc[sel[:, 1:]].all()), "not strictly ascending"
+    assert bool((ix[~sel] == -1).all()), "padding"
+    short = (klen <= k).view(T, 1) & sel
+    assert bool((ix == col)[short].all()), "short row takes every key"
+    assert bool(torch.isfinite(out).all()), "non-finite output"
+    assert bool(torch.isfinite(lse).all()), "non-finite lse"
+
+
+def test_prefill_64k_full(N):
+    # the call bench.py times for the 64K prefill: one dsa_forward over all
+    # 65,536 rows (128 chunks of 512 rows, query groups of 4)
+    import torch
+    from long_context_sparse_04_b200.workload import DeviceWorkload
+    cfg = I.CONFIGS["prefill_64k"]
+    sample = [0, 1, 2046, 2047, 2048, 9999, 30000, 45001, 65534, 65535]
+    inp = I.generate(cfg, threads=16)
+    wl = DeviceWorkload(inp)
+    out, lse, idx = wl.forward()
+    torch.cuda.synchronize()
+    assert wl.status(N.DSA_OP_FORWARD) == (0, -1)
+    ran = wl.kernels_ran(N.DSA_OP_FORWARD)
+    assert ran & N.DSA_KERNEL_INDEXER_TC and ran & N.DSA_KERNEL_TOPK and ran & N.DSA_KERNEL_MLA_TC
+    _check_selection_properties_device(inp["row_klen"], int(inp["topk"]), idx, out, lse)
+    s_out, s_lse, s_idx = (P.to_np(x[sample]) for x in (out, lse, idx))
+    del wl, out, lse, idx, inp
+    torch.cuda.empty_cache()
+    # the sampled rows alone, stage by stage: their scores for the oracle
+    # comparison; the selection must not depend on the batch
+    sub = I.generate(cfg, rows=sample, threads=16)
+    ws = DeviceWorkload(sub)
+    r_sc = ws.indexer()
+    r_idx = ws.topk_(r_sc)
+    torch.cuda.synchronize()
+    r_sc, r_idx = P.to_np(r_sc), P.to_np(r_idx)
+    assert np.array_equal(r_idx, s_idx), "selection depends on the batch"
+    P.check_rows(sub, range(len(sample)), r_sc, s_idx, s_out, s_lse)
 
 
 def test_prefill_64k_sampled_rows(N):
