@@ -23,10 +23,22 @@
 // rescale: the running max is only moved (and O rescaled) when a block's max
 // exceeds it by more than 8, so P stays <= 256.
 //
-// Roles per CTA (416 threads): warps 0-3 gather (cp.async, 16-byte pieces,
-// swizzled), warps 4-7 push the partial logits to the peer, warps 8-11 softmax
-// and epilogue (thread = head = TMEM lane), warp 12 TMEM allocation and
-// single-thread MMA issue.
+// Roles per CTA (896 threads, seven warpgroups):
+//   warp 0       TMEM allocation and single-thread MMA issue
+//   warps 1-15   gather: 16-byte cp.async pieces of the selected rows into a
+//                swizzled 3-stage ring.  A random 576-byte half row is a few
+//                sectors from each of many DRAM pages, so the gather is bound
+//                by the loads each warp keeps in flight: fifteen issuing warps
+//                keep ~3x more bytes in flight than four.
+//   warps 16-19  exchange: partial logits of block j to the peer while the
+//                softmax works on block j-1 (thread = head = TMEM lane)
+//   warps 20-27  softmax and epilogue: two warps per TMEM lane quarter, each
+//                taking 32 of the block's 64 keys of its 32 heads, so the
+//                per-block chain is half as long; the two halves agree on the
+//                row max through shared memory
+// The gather and MMA warpgroups give registers to the exchange and softmax
+// warpgroups (setmaxnreg): 4 x 128 x 48 + 3 x 128 x 104 = 64,512 registers,
+// the 896 threads x 72 the kernel is launched with (checked before launch).
 // TMEM: S double buffer (2 x 64 cols), P double buffer (2 x 32 cols of bf16x2),
 // O (256 cols).
 #include <cuda_bf16.h>
@@ -40,7 +52,15 @@ constexpr int kH = 128, kDC = 512, kDR = 64, kD = kDC + kDR;
 constexpr int kBlk = 64;
 constexpr int kNS = 3;
 constexpr int kMaxKeys = 2048;
-constexpr int kThreads = 32 * 13;
+constexpr int kGatherWarp0 = 1, kGatherWarps = 15;
+constexpr int kGatherThreads = 32 * kGatherWarps;       // 480
+constexpr int kExWarp0 = 16;                            // warps 16-19
+constexpr int kSmWarp0 = 20;                            // warps 20-27
+constexpr int kThreads = 32 * 28;                       // 896: seven warpgroups
+constexpr int kRegsLaunch = 72, kRegsLow = 48, kRegsHigh = 104;
+static_assert(4 * 128 * kRegsLow + 3 * 128 * kRegsHigh <= kThreads * kRegsLaunch,
+              "register split exceeds the launch's registers");
+static_assert(kThreads * kRegsLaunch <= 65536, "launch registers exceed the SM's");
 constexpr int kPieces = 36;                 // 16-byte pieces of one key's 288 dims per CTA
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -63,6 +83,8 @@ struct __align__(1024) MlaSmem {
   XTile sbuf;                               // this CTA's partial logits, bulk-copied to the peer
   int32_t rows[kMaxKeys];                   // physical cache row per selected key, -1 = none
   unsigned long long valid[kMaxKeys / kBlk];
+  float red_m[2][2][kH];                    // softmax halves: block max, [block parity][half][head]
+  float red_l[2][kH];                       // softmax halves: final sums
   uint64_t q_full, x_full, x_free;
   uint64_t kv_full[kNS], kv_empty[kNS];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
@@ -87,7 +109,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // 2^-64).  Error <= 2^-11 in the exponent (0.034% in the weight).  Encoding and
 // decoding use a float magic-number add, so no conversion instruction is needed.
 constexpr float kFix = 1024.f, kFixInv = 1.f / 1024.f, kMagic = 12582912.f;   // 1.5 * 2^23
-__device__ __forceinline__ float encode_partial(float (&z)[64], float c, uint32_t (&pk)[32]) {
+// Encodes row h of a partial logit tile (z, scaled here by c) into `x`: the
+// row max and eight swizzled 16-byte pieces of packed distances.
+__device__ __forceinline__ void encode_partial(float (&z)[64], float c, XTile& x, int h) {
   float pm[8];
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
@@ -97,12 +121,18 @@ __device__ __forceinline__ float encode_partial(float (&z)[64], float c, uint32_
   const float m = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                         fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t u0 = __float_as_uint(fminf((m - z[2 * i]) * kFix, 65535.f) + kMagic);
-    const uint32_t u1 = __float_as_uint(fminf((m - z[2 * i + 1]) * kFix, 65535.f) + kMagic);
-    pk[i] = __byte_perm(u0, u1, 0x5410);          // low 16 bits of each
+  for (int q = 0; q < 8; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = 4 * q + e;
+      const uint32_t u0 = __float_as_uint(fminf((m - z[2 * i]) * kFix, 65535.f) + kMagic);
+      const uint32_t u1 = __float_as_uint(fminf((m - z[2 * i + 1]) * kFix, 65535.f) + kMagic);
+      w[e] = __byte_perm(u0, u1, 0x5410);         // low 16 bits of each
+    }
+    x.d[h * 8 + (q ^ (h & 7))] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  return m;
+  x.m[h] = m;
 }
 // z of the two keys packed in w, given the row max m.
 __device__ __forceinline__ float2 decode_partial(uint32_t w, float m) {
@@ -116,11 +146,68 @@ __device__ __forceinline__ void tstamp(long long* tr, uint32_t rank, int ev, int
     tr[((int)rank * kTraceEvents + ev) * kTraceBlocks + j] = clock64();
 }
 
+__device__ __forceinline__ void setmaxnreg_inc_high() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+}
+__device__ __forceinline__ void setmaxnreg_dec_low() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+}
+
+// ------------------------------------------------------------ MMA issuer (warp 0, lane 0)
+__device__ __forceinline__ void mma_role(MlaSmem& S, const MlaArgs& a, uint32_t tmem, int nblk,
+                                         uint32_t rank) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0 && nblk > 0) {
+    constexpr uint32_t idesc_s = idesc_bf16(kBlk, false);
+    constexpr uint32_t idesc_pv = idesc_bf16(256, true);
+    bool ok = mbar_wait(&S.q_full, 0, a.status, 31);
+    fence_proxy_async_smem();
+    const uint32_t qa = smem_u32(S.q[0]), qra = smem_u32(S.q_rope);
+    for (int j = 0; ok && j <= nblk; ++j) {
+      if (j < nblk) {
+        const int st = j % kNS, b = j & 1;
+        if (!(ok = mbar_wait(&S.kv_full[st], (j / kNS) & 1, a.status, 32))) break;
+        fence_proxy_async_smem();           // gathered (generic-proxy) writes -> tensor cores
+        if (!(ok = mbar_wait(&S.s_free[b], ((j >> 1) & 1) ^ 1, a.status, 33))) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(S.kv[st][0]), kra = smem_u32(S.kv_rope[st]);
+        const uint32_t d = tmem + kColS + b * 64;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(d, sdesc_sw128(qa + ch * kH * 128 + 32 * kk, 16, 1024),
+                     sdesc_sw128(ka + ch * kBlk * 128 + 32 * kk, 16, 1024), idesc_s,
+                     (ch | kk) != 0);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_bf16(d, sdesc_sw64(qra + 32 * kk, 512), sdesc_sw64(kra + 32 * kk, 512), idesc_s, 1);
+        mma_commit(&S.s_full[b]);
+        tstamp(a.trace, rank, 2, j);
+      }
+      if (j >= 1) {
+        const int jj = j - 1, st = jj % kNS, b = jj & 1;
+        if (!(ok = mbar_wait(&S.p_full[b], (jj >> 1) & 1, a.status, 34))) break;
+        tc_fence_after();
+        const uint32_t va = smem_u32(S.kv[st][0]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ts(tmem + kColO, tmem + kColP + b * 32 + kk * 8,
+                      sdesc_sw128(va + kk * 16 * 128, kBlk * 128, 1024), idesc_pv,
+                      (jj > 0 || kk > 0));
+        mma_commit(&S.kv_empty[st]);
+        mma_commit(&S.pv_done[b]);
+        tstamp(a.trace, rank, 3, jj);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys_per_split) {
   extern __shared__ __align__(1024) uint8_t smraw[];
   MlaSmem& S = *reinterpret_cast<MlaSmem*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                            ~uintptr_t(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
   const int unit = blockIdx.x >> 1;
   const int t = unit / a.splits, sp = unit % a.splits;
@@ -132,20 +219,23 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   // writes any of them (and triggers its dependents early) is complete and
   // visible first.
   if (threadIdx.x == 0) {
-    mbar_init(&S.q_full, 128);
+    mbar_init(&S.q_full, kGatherThreads);
     mbar_init(&S.x_full, 1);                 // armed by this CTA, completed by the peer's copy
     mbar_init(&S.x_free, 1);                 // the peer's receive buffer is free
-    for (int i = 0; i < kNS; ++i) { mbar_init(&S.kv_full[i], 128); mbar_init(&S.kv_empty[i], 1); }
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&S.kv_full[i], kGatherThreads);
+      mbar_init(&S.kv_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_free[i], 256);         // exchange + softmax warpgroups
-      mbar_init(&S.p_full[i], 128);
+      mbar_init(&S.s_free[i], 128 + 256);   // exchange + softmax warpgroups
+      mbar_init(&S.p_full[i], 256);         // softmax warpgroups
       mbar_init(&S.pv_done[i], 1);
     }
     fence_mbar_init();
   }
   __syncwarp();
-  if (warp == 12) {
+  if (warp == 0) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -158,12 +248,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   const int nblk = (nvalid + kBlk - 1) / kBlk;
   const int seq = a.row_seq[t];
   if (threadIdx.x == 0 && nblk > 0) mbar_expect_tx(&S.x_full, kXBytes);   // arm the first transfer
+  const bool gather_warp = warp >= kGatherWarp0 && warp < kGatherWarp0 + kGatherWarps;
+  const int g = threadIdx.x - 32 * kGatherWarp0;          // gather thread index (0..479)
   // Q first: its pieces land while the selection is resolved below (the
   // gather warps arrive on q_full for them once the barrier init is visible)
-  if (warp < 4 && nblk > 0) {
+  if (gather_warp && nblk > 0) {
     const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
-    for (int i = 0; i < kPieces; ++i) {
-      const int qi = i * 128 + threadIdx.x;
+    for (int qi = g; qi < kH * kPieces; qi += kGatherThreads) {
       const int h = qi / kPieces, c = qi - h * kPieces;
       if (c < 32) {
         cp_async_16(S.q[c >> 3] + sw128_off(h, c & 7), qrow + h * kD + 256 * rank + 8 * c);
@@ -210,19 +301,21 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   tc_fence_after();
   cluster_sync();   // the peer's barriers are initialised before any remote arrive
   const uint32_t tmem = S.tmem_base;
-
-  if (warp < 4) {
-    // ------------------------------------------------------------ gather (128 threads)
-    const int tid = threadIdx.x;
-    if (nblk > 0) {
+  // Registers: the gather / MMA warpgroups (0-3) give theirs to the exchange
+  // and softmax warpgroups (4-6).  Each warpgroup executes one setmaxnreg, at
+  // the head of its role's branch.
+  if (warp < kExWarp0) {
+    setmaxnreg_dec_low();
+    if (warp == 0) {
+      mma_role(S, a, tmem, nblk, rank);
+    } else if (nblk > 0) {
+    // ------------------------------------------------------------ gather (480 threads)
       cp_async_mbar_arrive(&S.q_full);        // arrives when this thread's Q pieces land
       const __nv_bfloat16* lat = static_cast<const __nv_bfloat16*>(a.latent);
-      bool alive = true;
       for (int j = 0; j < nblk; ++j) {
         const int st = j % kNS;
-        if (!mbar_wait(&S.kv_empty[st], ((j / kNS) & 1) ^ 1, a.status, 21)) { alive = false; break; }
-        for (int i = 0; i < (kBlk * kPieces) / 128; ++i) {
-          const int qi = i * 128 + tid;
+        if (!mbar_wait(&S.kv_empty[st], ((j / kNS) & 1) ^ 1, a.status, 21)) break;
+        for (int qi = g; qi < kBlk * kPieces; qi += kGatherThreads) {
           const int key = qi / kPieces, c = qi - key * kPieces;
           const int row = S.rows[j * kBlk + key];
           const __nv_bfloat16* src = lat + (int64_t)(row < 0 ? 0 : row) * kD +
@@ -236,22 +329,22 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         cp_async_mbar_arrive(&S.kv_full[st]);
       }
       cp_async_wait_all();
-      (void)alive;
     }
-  } else if (warp < 8) {
+  } else if (warp < kSmWarp0) {
+    setmaxnreg_inc_high();
     // ------------------------------------------------------------ exchange (128 threads)
     // Copies this CTA's partial logits of block j to the peer with one bulk copy
-    // while the softmax warpgroup is still working on block j-1.  A wait that
+    // while the softmax warpgroups are still working on block j-1.  A wait that
     // times out only marks the warpgroup dead: the named barriers stay uniform.
-    const int h = threadIdx.x - 128;                          // head = TMEM lane
+    const int h = threadIdx.x - 32 * kExWarp0;                // head = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const float c = a.sm_scale * kLog2e;
     bool dead = false;
     for (int j = 0; j < nblk; ++j) {
       const int b = j & 1;
       float z[64];
-      uint32_t pk[32];
-      float m = 0.f;
+      if (h == 0 && j > 0) bulk_wait_read0();               // the previous copy has left sbuf
+      named_bar_sync(2, 128);
       dead = dead || !mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 22);
       if (!dead) {
         tc_fence_after();
@@ -260,15 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&S.s_free[b]);
-        m = encode_partial(z, c, pk);
-      }
-      if (h == 0 && j > 0) bulk_wait_read0();               // the previous copy has left sbuf
-      named_bar_sync(2, 128);
-      if (!dead) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          S.sbuf.d[h * 8 + (q ^ (h & 7))] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        S.sbuf.m[h] = m;
+        encode_partial(z, c, S.sbuf, h);
       }
       fence_proxy_async_smem();                              // sbuf writes -> async copy engine
       named_bar_sync(2, 128);
@@ -280,9 +365,15 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       }
     }
     if (h == 0) bulk_wait_read0();
-  } else if (warp < 12) {
-    // ------------------------------------------------------------ softmax / output (128 threads)
-    const int h = threadIdx.x - 256;                          // head = TMEM lane
+  } else {
+    setmaxnreg_inc_high();
+    // ------------------------------------------------------------ softmax / output (256 threads)
+    // Thread (half, h): head h (= TMEM lane), keys [32 half, 32 half + 32) of
+    // every block, value dims [128 half, 128 half + 128) of this CTA's 256 in
+    // the epilogue.  Both halves take the same rescale decisions: they use the
+    // same block max (exchanged through red_m) and the same running max.
+    const int sidx = threadIdx.x - 32 * kSmWarp0;             // 0..255
+    const int half = sidx >> 7, h = sidx & 127;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const float c = a.sm_scale * kLog2e;
     float m_used = -INFINITY, l = 0.f;
@@ -293,54 +384,57 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       const int b = j & 1;
       dead = dead || !mbar_wait(&S.s_full[b], (j >> 1) & 1, a.status, 28);
       tc_fence_after();
-      if (h == 0) tstamp(a.trace, rank, 4, j);
-      float s[64];
-      tmem_ld32(tmem + lane_off + kColS + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(tmem + lane_off + kColS + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      if (sidx == 0) tstamp(a.trace, rank, 4, j);
+      float s[32];
+      tmem_ld32(tmem + lane_off + kColS + b * 64 + 32 * half, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&S.s_free[b]);
-      // z = c * S_own (exact) + the peer's partial (decoded).  The two
-      // CTAs see the same sum up to that rounding; each keeps its own softmax
-      // state (m, l), used for its own half of the value dims.
-#pragma unroll
-      for (int i = 0; i < 64; ++i) s[i] *= c;
+      // z = c * S_own (exact) + the peer's partial (decoded).  The two CTAs see
+      // the same sum up to that rounding; each keeps its own softmax state
+      // (m, l), used for its own half of the value dims.
       dead = dead || !mbar_wait_cluster(&S.x_full, j & 1, a.status, 24);
-      if (h == 0) tstamp(a.trace, rank, 5, j);
-      const float m_peer = S.xbuf.m[h];
+      if (sidx == 0) tstamp(a.trace, rank, 5, j);
+      {
+        const float m_peer = S.xbuf.m[h];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 w4 = S.xbuf.d[h * 8 + (q ^ (h & 7))];
-        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w4 = S.xbuf.d[h * 8 + ((4 * half + q) ^ (h & 7))];
+          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = decode_partial(w[e], m_peer);
-          s[8 * q + 2 * e] += f.x;
-          s[8 * q + 2 * e + 1] += f.y;
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = decode_partial(w[e], m_peer);
+            s[8 * q + 2 * e] = fmaf(s[8 * q + 2 * e], c, f.x);
+            s[8 * q + 2 * e + 1] = fmaf(s[8 * q + 2 * e + 1], c, f.y);
+          }
         }
       }
-      if (h == 0) tstamp(a.trace, rank, 0, j);
-      if (named_bar_or(3, 128, dead)) { dead = true; break; }   // whole tile read, all alive
-      if (h == 0) {
+      if (sidx == 0) tstamp(a.trace, rank, 0, j);
+      // masked (only partial blocks) logits in the log2 domain; this half's max
+      const unsigned long long mask = S.valid[j] >> (32 * half);
+      if ((uint32_t)mask != 0xFFFFFFFFu) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (!((mask >> i) & 1ull)) s[i] = -INFINITY;
+      }
+      float pm[8];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pm[i & 7] = (i < 8) ? s[i] : fmaxf(pm[i & 7], s[i]);
+      const float mh = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      S.red_m[b][half][h] = mh;
+      // every softmax thread has read xbuf and published its half's max; all alive
+      if (named_bar_or(3, 256, dead)) { dead = true; break; }
+      if (sidx == 0) {
         if (j + 1 < nblk) mbar_expect_tx(&S.x_full, kXBytes);   // arm the next transfer first
         // then free the buffer: every thread's reads of it were consumed before
         // the barrier above, so the arrive needs no release ordering
         mbar_arrive_cluster_relaxed(&S.x_free, peer);
       }
-      if (h == 0) tstamp(a.trace, rank, 1, j);
-      // masked (only partial blocks), scaled logits in the log2 domain; block max
-      const unsigned long long mask = S.valid[j];
-      if (mask != ~0ull) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (!((mask >> i) & 1ull)) s[i] = -INFINITY;
-      }
-      float pm[8];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) pm[i & 7] = (i < 8) ? s[i] : fmaxf(pm[i & 7], s[i]);
-      const float mb = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      // lazy rescale (warp-uniform because tcgen05.ld/st are warp-collective)
+      if (sidx == 0) tstamp(a.trace, rank, 1, j);
+      const float mb = fmaxf(mh, S.red_m[b][half ^ 1][h]);
+      // lazy rescale (warp-uniform because tcgen05.ld/st are warp-collective;
+      // both halves of a lane quarter decide alike)
       const bool need = mb > m_used + kRescale;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? mb : m_used;
@@ -349,13 +443,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
           dead = dead || !mbar_wait(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.status, 25);
           tc_fence_after();
 #pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_off + kColO + 32 * cc, o);
+            const uint32_t col = tmem + lane_off + kColO + 128 * half + 32 * cc;
+            tmem_ld32(col, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_off + kColO + 32 * cc, o);
+            tmem_st32(col, o);
           }
           tmem_wait_st();
         }
@@ -365,54 +460,58 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       // p = 2^(s - m); a masked key (s = -inf) gives 0.  While no key of the row
       // has been visible, every s is -inf and m is taken as 0.
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t p2[32];
+      uint32_t p2[16];
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float p0 = ex2_approx(s[2 * i] - mu);
         const float p1 = ex2_approx(s[2 * i + 1] - mu);
         ls[i & 3] += p0 + p1;
         p2[i] = pack_bf16x2(p0, p1);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      if (h == 0) tstamp(a.trace, rank, 7, j);
+      if (sidx == 0) tstamp(a.trace, rank, 7, j);
       // P buffer b is free once the PV of block j-2 is done
       dead = dead || !mbar_wait(&S.pv_done[b], ((j >> 1) & 1) ^ 1, a.status, 26);
       tc_fence_after();
-      tmem_st32(tmem + lane_off + kColP + b * 32, p2);
+      tmem_st16(tmem + lane_off + kColP + b * 32 + 16 * half, p2);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&S.p_full[b]);
-      if (h == 0) tstamp(a.trace, rank, 6, j);
+      if (sidx == 0) tstamp(a.trace, rank, 6, j);
     }
-    // ---- output
+    // ---- output: this CTA's value dims [128 half, 128 half + 128) of head h
     const int64_t ro = ((int64_t)t * kH + h);
     if (!dead && nblk > 0) {
       dead = !mbar_wait(&S.pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, 27);
       tc_fence_after();
     }
+    // the row's sum over both key halves
+    S.red_l[half][h] = l;
+    named_bar_sync(4, 256);
+    const float lt = S.red_l[0][h] + S.red_l[1][h];
     const bool have = __all_sync(0xffffffffu, !dead) && nblk > 0;
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
 #pragma unroll 1
-    for (int cc = 0; cc < 8; ++cc) {
+    for (int cc = 0; cc < 4; ++cc) {
       uint32_t o[32];
       if (have) {
-        tmem_ld32(tmem + lane_off + kColO + 32 * cc, o);
+        tmem_ld32(tmem + lane_off + kColO + 128 * half + 32 * cc, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
+      const int dim0 = 256 * (int)rank + 128 * half + 32 * cc;
       if (a.splits > 1) {
         float4* dst = reinterpret_cast<float4*>(
-            a.part_o + (((int64_t)t * a.splits + sp) * kH + h) * kDC + 256 * rank + 32 * cc);
+            a.part_o + (((int64_t)t * a.splits + sp) * kH + h) * kDC + dim0);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
                                __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
       } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ro * kDC +
-                                              256 * rank + 32 * cc);
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ro * kDC + dim0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float* f = reinterpret_cast<const float*>(&o[8 * i]);
@@ -421,65 +520,19 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         }
       }
     }
-    if (a.splits > 1 || rank == 0) {
+    if (half == 0 && (a.splits > 1 || rank == 0)) {
       if (a.splits > 1) {
         reinterpret_cast<float2*>(a.part_ml)[(((int64_t)t * a.splits + sp) * 2 + rank) * kH + h] =
-            make_float2(m_used, l);
+            make_float2(m_used, lt);
       } else if (a.lse) {
-        a.lse[ro] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nblk > 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(kBlk, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(256, true);
-      bool ok = mbar_wait(&S.q_full, 0, a.status, 31);
-      fence_proxy_async_smem();
-      const uint32_t qa = smem_u32(S.q[0]), qra = smem_u32(S.q_rope);
-      for (int j = 0; ok && j <= nblk; ++j) {
-        if (j < nblk) {
-          const int st = j % kNS, b = j & 1;
-          if (!(ok = mbar_wait(&S.kv_full[st], (j / kNS) & 1, a.status, 32))) break;
-          fence_proxy_async_smem();           // gathered (generic-proxy) writes -> tensor cores
-          if (!(ok = mbar_wait(&S.s_free[b], ((j >> 1) & 1) ^ 1, a.status, 33))) break;
-          tc_fence_after();
-          const uint32_t ka = smem_u32(S.kv[st][0]), kra = smem_u32(S.kv_rope[st]);
-          const uint32_t d = tmem + kColS + b * 64;
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(d, sdesc_sw128(qa + ch * kH * 128 + 32 * kk, 16, 1024),
-                       sdesc_sw128(ka + ch * kBlk * 128 + 32 * kk, 16, 1024), idesc_s,
-                       (ch | kk) != 0);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_bf16(d, sdesc_sw64(qra + 32 * kk, 512), sdesc_sw64(kra + 32 * kk, 512), idesc_s, 1);
-          mma_commit(&S.s_full[b]);
-          tstamp(a.trace, rank, 2, j);
-        }
-        if (j >= 1) {
-          const int jj = j - 1, st = jj % kNS, b = jj & 1;
-          if (!(ok = mbar_wait(&S.p_full[b], (jj >> 1) & 1, a.status, 34))) break;
-          tc_fence_after();
-          const uint32_t va = smem_u32(S.kv[st][0]);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem + kColO, tmem + kColP + b * 32 + kk * 8,
-                        sdesc_sw128(va + kk * 16 * 128, kBlk * 128, 1024), idesc_pv,
-                        (jj > 0 || kk > 0));
-          mma_commit(&S.kv_empty[st]);
-          mma_commit(&S.pv_done[b]);
-          tstamp(a.trace, rank, 3, jj);
-        }
+        a.lse[ro] = lt > 0.f ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   cluster_sync();   // no remote access to this CTA's shared memory is still pending
-  if (warp == 12) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -537,12 +590,41 @@ size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits) {
   return (size_t)num_rows * splits * n_heads * (d_c * sizeof(float) + 4 * sizeof(float));
 }
 
+static_assert(sizeof(MlaSmem) + 1024 <= 227 * 1024, "shared memory of the attention kernel");
+
+// The kernel moves registers between warpgroups (setmaxnreg): the increases
+// wait until the decreases have returned enough registers, which needs the
+// launch to hold exactly the register budget the split was sized for.  A
+// build whose register count differs is refused instead of launched.
+dsa_status check_register_split() {
+  static std::atomic<int> ok[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_error("no current CUDA device");
+    return DSA_ERR_CUDA;
+  }
+  if (dev >= 0 && dev < kMaxDevices && ok[dev].load(std::memory_order_acquire) == 1) return DSA_OK;
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, mla_tc_kernel) != cudaSuccess) {
+    set_error("cudaFuncGetAttributes(mla_tc_kernel) failed");
+    return DSA_ERR_CUDA;
+  }
+  if (fa.numRegs != kRegsLaunch) {
+    set_error("mla_tc_kernel built with %d registers per thread; its warpgroup register split "
+              "needs exactly %d", fa.numRegs, kRegsLaunch);
+    return DSA_ERR_UNSUPPORTED;
+  }
+  if (dev >= 0 && dev < kMaxDevices) ok[dev].store(1, std::memory_order_release);
+  return DSA_OK;
+}
+
 dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
   const size_t smem = sizeof(MlaSmem) + 1024;
   static std::atomic<bool> attr[kMaxDevices] = {};
   if (dsa_status st = set_smem_limit_once(reinterpret_cast<const void*>(mla_tc_kernel), smem, attr))
     return st;
+  if (dsa_status st = check_register_split()) return st;
   const int keys_per_split = (int)(ceil_div64(ceil_div64(a.topk, a.splits), kBlk) * kBlk);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.num_rows * a.splits * 2));
