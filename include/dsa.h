@@ -73,10 +73,19 @@ typedef enum {
 
 /* Which kernels to run.  AUTO picks the tensor-core kernels (tcgen05) for the
  * FP8 indexer with H_I*group <= 256, d_I = 128, and for bf16 MLA with
- * H = 128, d_c = 512, d_r = 64; everything else runs the SIMT kernels. */
+ * H = 128, d_c = 512, d_r = 64; everything else runs the SIMT kernels.  With
+ * AUTO, dsa_decode_step and dsa_forward fuse the indexer and top-k when the
+ * tensor-core indexer runs and q_group <= 2: the indexer's epilogue also
+ * builds each row's histogram of its scores' top 12 order-preserving key bits
+ * (the first pass of the radix selection), and top-k starts from it
+ * ("DeepSeek Sparse Attention DSA Architecture Guide", section "Stage 1: The
+ * Lightning Indexer", item "Separable Streaming Top-k": the selection is
+ * folded into the indexer's pass).  STAGED runs the same tensor-core kernels
+ * without that fusion (top-k builds its own histogram), as dsa_topk does. */
 typedef enum {
   DSA_ALGO_AUTO = 0,
-  DSA_ALGO_SIMT = 1
+  DSA_ALGO_SIMT = 1,
+  DSA_ALGO_STAGED = 2
 } dsa_algo;
 
 /* Problem dimensions. */
@@ -148,7 +157,12 @@ int32_t dsa_version(void);
  * DSA_OP_CACHE_APPEND needs only the status block; `rows` may be NULL for it. */
 size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op);
 
-/* Zero the device status word at the head of `ws` (async on stream). */
+/* Zero the workspace `ws` (ws_bytes bytes, async on stream): the device status
+ * word at its head and, for dsa_decode_step and dsa_forward, the per-row
+ * score histograms of the fused indexer -> top-k, which every top-k leaves
+ * zeroed for the next call.  Call it once before the first use of a
+ * workspace, and again after a call that recorded a device error (a call cut
+ * short may leave histograms behind). */
 dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /* Synchronise `stream`, copy the device status word of `ws` to *status_out

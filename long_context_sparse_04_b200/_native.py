@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA = 0, 1, 2, 3
 DSA_ERR_OUT_OF_RANGE, DSA_ERR_TIMEOUT, DSA_ERR_WORKSPACE = 4, 5, 6
 DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
-DSA_ALGO_AUTO, DSA_ALGO_SIMT = 0, 1
+DSA_ALGO_AUTO, DSA_ALGO_SIMT, DSA_ALGO_STAGED = 0, 1, 2
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE_STEP, DSA_OP_FORWARD = range(5)
 DSA_OP_CACHE_APPEND = 5
 DSA_KERNEL_INDEXER_SIMT, DSA_KERNEL_INDEXER_TC, DSA_KERNEL_TOPK = 0x01, 0x02, 0x04

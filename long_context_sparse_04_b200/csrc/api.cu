@@ -88,7 +88,8 @@ dsa_status check_dims(const dsa_dims* d) {
   CHECK_ARG(d->topk >= 1 && d->topk <= 2048, "topk %d outside [1, 2048]", d->topk);
   CHECK_ARG(d->idx_dtype == DSA_FP8_E4M3 || d->idx_dtype == DSA_F32, "idx_dtype must be e4m3 or f32");
   CHECK_ARG(d->mla_dtype == DSA_BF16 || d->mla_dtype == DSA_F32, "mla_dtype must be bf16 or f32");
-  CHECK_ARG(d->algo == DSA_ALGO_AUTO || d->algo == DSA_ALGO_SIMT, "unknown algo");
+  CHECK_ARG(d->algo == DSA_ALGO_AUTO || d->algo == DSA_ALGO_SIMT || d->algo == DSA_ALGO_STAGED,
+            "unknown algo");
   CHECK_ARG(d->sm_scale > 0.f, "sm_scale must be > 0");
   if (d->d_idx % 4 != 0 || (d->d_c + d->d_r) % 8 != 0) {
     set_error("d_idx must be a multiple of 4 and d_c + d_r a multiple of 8");
@@ -168,6 +169,7 @@ struct WsPlan {
   size_t scores = 0, scores_bytes = 0;
   size_t idx = 0, idx_bytes = 0;
   size_t mla = 0, mla_bytes = 0;
+  size_t hist = 0, hist_bytes = 0;
   size_t total = 0;
   int64_t ld = 0;
   int chunk_rows = 0;
@@ -203,6 +205,13 @@ WsPlan plan(const dsa_dims* d, const dsa_rows* r, dsa_op op) {
     p.mla = off;
     p.mla_bytes = align_up(mla_ws_bytes(rows, d->n_heads, d->d_c, p.splits));
     off += p.mla_bytes;
+  }
+  // per-row score histograms of the fused indexer -> top-k (query groups of
+  // at most 2 rows); zeroed by dsa_workspace_init and left zeroed by each top-k
+  if (need_buf && r->q_group <= 2) {
+    p.hist = off;
+    p.hist_bytes = align_up((size_t)rows * 4096 * sizeof(uint32_t));
+    off += p.hist_bytes;
   }
   p.total = off;
   return p;
@@ -250,9 +259,16 @@ IndexerArgs indexer_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* 
 
 dsa_status run_indexer(const dsa_dims* d, IndexerArgs& a, void* ws, const WsPlan& p,
                        cudaStream_t s) {
-  if (d->algo == DSA_ALGO_AUTO && indexer_tc_supported(a))
+  if (d->algo != DSA_ALGO_SIMT && indexer_tc_supported(a))
     return launch_indexer_tc(a, at(ws, p.indexer), p.indexer_bytes, s);
   return launch_indexer_simt(a, s);
+}
+
+// The fused indexer -> top-k: the indexer builds each row's histogram of its
+// scores' top 12 key bits, and top-k starts from it.
+uint32_t* fused_hist(const dsa_dims* d, const IndexerArgs& ia, void* ws, const WsPlan& p) {
+  if (d->algo != DSA_ALGO_AUTO || p.hist_bytes == 0 || !indexer_tc_hist_supported(ia)) return nullptr;
+  return reinterpret_cast<uint32_t*>(at(ws, p.hist));
 }
 
 MlaArgs mla_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c, const void* q,
@@ -282,7 +298,7 @@ MlaArgs mla_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c, const
 }
 
 dsa_status run_mla(const dsa_dims* d, MlaArgs& a, cudaStream_t s) {
-  if (d->algo == DSA_ALGO_AUTO && mla_tc_supported(a)) return launch_mla_tc(a, s);
+  if (d->algo != DSA_ALGO_SIMT && mla_tc_supported(a)) return launch_mla_tc(a, s);
   return launch_mla_simt(a, s);
 }
 
@@ -352,7 +368,7 @@ size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op)
 
 dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream) {
   if (check_ws(ws, ws_bytes, kStatusBytes) != DSA_OK) return DSA_ERR_WORKSPACE;
-  if (cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream) != cudaSuccess) {
+  if (cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) != cudaSuccess) {
     set_error("cudaMemsetAsync failed");
     return DSA_ERR_CUDA;
   }
@@ -541,6 +557,7 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   float* scores = dbg_scores ? dbg_scores : reinterpret_cast<float*>(at(ws, p.scores));
   int32_t* idx = dbg_idx ? dbg_idx : reinterpret_cast<int32_t*>(at(ws, p.idx));
   IndexerArgs ia = indexer_args(dims, rows, cache, q_idx, q_scale, w, scores, p.ld, ws, p);
+  ia.hist = fused_hist(dims, ia, ws, p);
   stage_event(0, s);
   if ((st = run_indexer(dims, ia, ws, p, s))) return st;
   stage_event(1, s);
@@ -553,6 +570,7 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   ta.idx = idx;
   ta.status = reinterpret_cast<DeviceStatus*>(ws);
   ta.trace = trace_buffer();
+  ta.hist = ia.hist;
   if ((st = launch_topk(ta, rows->max_klen, s))) return st;
   stage_event(2, s);
   MlaArgs ma = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
@@ -599,6 +617,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     float* ll = lse ? lse + (size_t)r0 * H : nullptr;
     int32_t* idx = idx_out ? idx_out + (size_t)r0 * dims->topk : idx_ws;
     IndexerArgs ia = indexer_args(dims, &cr, cache, qi, qs, wr, scores, p.ld, ws, p);
+    ia.hist = fused_hist(dims, ia, ws, p);
     if ((st = run_indexer(dims, ia, ws, p, s))) return st;
     TopkArgs ta{};
     ta.num_rows = n;
@@ -608,7 +627,8 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     ta.topk = dims->topk;
     ta.idx = idx;
     ta.status = reinterpret_cast<DeviceStatus*>(ws);
-  ta.trace = trace_buffer();
+    ta.trace = trace_buffer();
+    ta.hist = ia.hist;
     if ((st = launch_topk(ta, rows->max_klen, s))) return st;
     MlaArgs ma = mla_args(dims, &cr, cache, qq, idx, oo, ll, ws, p);
     if ((st = run_mla(dims, ma, s))) return st;

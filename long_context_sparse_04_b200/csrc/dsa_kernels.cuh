@@ -24,6 +24,7 @@ struct IndexerArgs {
   int num_seqs;
   DeviceStatus* status;
   int32_t* tile_offsets;      // workspace: [n_groups + 1] exclusive scan of key tiles
+  uint32_t* hist;             // [num_rows, 4096] score-key histograms (zeroed), or null
 };
 
 struct TopkArgs {
@@ -35,6 +36,8 @@ struct TopkArgs {
   int32_t* idx;               // [T, topk]
   DeviceStatus* status;
   long long* trace;           // profiling stamps or null
+  uint32_t* hist;             // [T, 4096] histograms of the scores' top 12 key bits from the
+                              // indexer (read, then zeroed), or null: top-k builds its own
 };
 
 struct MlaArgs {
@@ -88,6 +91,8 @@ dsa_status launch_indexer_simt(const IndexerArgs& a, cudaStream_t stream);
 dsa_status launch_indexer_tc(const IndexerArgs& a, void* ws_tail, size_t ws_tail_bytes,
                              cudaStream_t stream);
 bool indexer_tc_supported(const IndexerArgs& a);
+// The indexer builds the rows' score histograms for top-k (fused path).
+bool indexer_tc_hist_supported(const IndexerArgs& a);
 size_t indexer_ws_bytes(int num_rows, int q_group);
 
 dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream);

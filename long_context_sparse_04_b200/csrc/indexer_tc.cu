@@ -33,6 +33,7 @@
 //               of the accumulator (lane = key), ReLU, head-weighted sum with w'
 //               (packed fp32x2 FMAs), times the key's scale, coalesced store.
 // The L x H_I per-head score tensor lives only in TMEM.
+#include <cstddef>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -47,7 +48,9 @@ constexpr int kHI = 64;
 constexpr int kEpiWarps = 16;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 2048;
-constexpr int kMaxCtaTiles = 512;
+// At most 511 tiles per CTA: a row's key count inside one CTA then stays below
+// 65,536, so the shared-memory score histogram can keep 16-bit counters.
+constexpr int kMaxCtaTiles = 511;
 constexpr int kKeyTileBytes = kTileKeys * kDI;   // 16 KB
 // Key-scale slots: the producer writes tile j's scales into slot j % 16 when it
 // fills the tile's key stage, and the epilogue reads them before it releases
@@ -57,9 +60,19 @@ constexpr int kKeyTileBytes = kTileKeys * kDI;   // 16 KB
 // (10 + 4, or 6 + 2) keeps a slot from being overwritten before it is read.
 constexpr int kScaleSlots = 16;
 
-// Key-tile stages in flight: as many as shared memory allows beside the queries.
+// Key-tile stages in flight: as many as shared memory allows beside the
+// queries (and, for NQ <= 2, the score histograms).
 template <int NQ>
-constexpr int num_stages() { return NQ <= 2 ? 10 : 6; }
+constexpr int num_stages() { return NQ <= 2 ? 8 : 6; }
+
+// Score histograms (NQ <= 2): for the first hist_slots() groups of a CTA's
+// range, per query row of the group, 4096 bins of the top 12 bits of the
+// order-preserving key of each score, two 16-bit counters per word.
+constexpr int kHistBins = 4096;
+template <int NQ>
+constexpr int hist_slots() { return NQ <= 2 ? 4 / NQ : 0; }
+template <int NQ>
+constexpr int hist_words() { return NQ <= 2 ? 4 * kHistBins / 2 : 4; }
 
 // TMEM accumulators per CTA: four of N columns when they fit in 512, else two.
 template <int NQ>
@@ -71,7 +84,8 @@ struct __align__(1024) IdxSmem {
   uint8_t q[2][NQ * kHI * kDI];
   float wq[kEpiWarps][kHI];                             // per epilogue warp: w' of its heads
   float kscale[kScaleSlots][kTileKeys];                 // key scales of tile j in slot j % kScaleSlots
-  int32_t tile_row[kMaxCtaTiles][2];                    // physical row of each 64-key half, -1: none
+  uint32_t hist[hist_words<NQ>()];                      // [slot][query of group][bin / 2]
+  alignas(16) int32_t tile_row[kMaxCtaTiles][2];        // physical row of each 64-key half, -1: none
   int32_t tile_info[kMaxCtaTiles];                      // group << 2 | last tile of group << 1 | first
   int32_t tile_off[kMaxGroups + 1];
   int32_t scan_tmp[kThreads / 32];
@@ -80,6 +94,15 @@ struct __align__(1024) IdxSmem {
   uint64_t acc_empty[4];
   uint32_t tmem_base;
 };
+
+// every member the kernel reads as a vector or fills with cp.async sits on a
+// 16-byte boundary (tile_row is read as int2, kscale filled 16 bytes at a time)
+static_assert(offsetof(IdxSmem<1>, tile_row) % 16 == 0 && offsetof(IdxSmem<2>, tile_row) % 16 == 0 &&
+                  offsetof(IdxSmem<4>, tile_row) % 16 == 0, "tile_row alignment");
+static_assert(offsetof(IdxSmem<1>, kscale) % 16 == 0 && offsetof(IdxSmem<2>, kscale) % 16 == 0 &&
+                  offsetof(IdxSmem<4>, kscale) % 16 == 0, "kscale alignment");
+static_assert(offsetof(IdxSmem<1>, wq) % 16 == 0 && offsetof(IdxSmem<2>, wq) % 16 == 0 &&
+                  offsetof(IdxSmem<4>, wq) % 16 == 0, "wq alignment");
 
 struct TcArgs {
   long long* trace;           // profiling stamps (CTA 0, first 32 tiles) or null
@@ -94,6 +117,7 @@ struct TcArgs {
   CacheMap map;
   float* scores;
   int64_t ld;
+  uint32_t* hist;             // [num_rows, 4096] score-key histograms to add to, or null
   DeviceStatus* status;
 };
 
@@ -251,8 +275,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       }
     }
   }
+  constexpr int kHistSlots = hist_slots<NQ>();
+  const bool use_hist = kHistSlots > 0 && a.hist != nullptr;
+  if (use_hist)
+    for (int i = threadIdx.x; i < hist_words<NQ>(); i += kThreads) S.hist[i] = 0u;
   __syncthreads();
   const bool run = ntile > 0 && ntile <= kMaxCtaTiles;
+  // the group of the CTA's first tile: histogram slot of group g is g - g_first
+  int g_first = 0;
+  if (run) {
+    TileIter it0;
+    it0.start(S.tile_off, a.n_groups, t_begin);
+    g_first = it0.g;
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -450,7 +485,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       }
       const float sum = ((lo[0] + hi[0]) + (lo[1] + hi[1])) + ((lo[2] + hi[2]) + (lo[3] + hi[3]));
       const int s = it.kt * kTileKeys + row_in_tile;
-      if (!dead && s < klen) a.scores[(int64_t)(it.g * NQ + qi) * a.ld + s] = sum * ks;
+      const float score = sum * ks;
+      if (!dead && s < klen) {
+        a.scores[(int64_t)(it.g * NQ + qi) * a.ld + s] = score;
+        if (use_hist) {
+          // the first selection pass of top-k, done here: the bin of this score
+          const uint32_t bin = float_key(score) >> 20;
+          const int slot = it.g - g_first;
+          if (slot < kHistSlots)
+            atomicAdd(&S.hist[(slot * NQ + qi) * (kHistBins / 2) + (bin >> 1)], 1u << (16 * (bin & 1)));
+          else
+            atomicAdd(&a.hist[(int64_t)(it.g * NQ + qi) * kHistBins + bin], 1u);
+        }
+      }
       if (threadIdx.x == 64) istamp(a.trace, 7, j);
       for (int k = 0; k < NSET; ++k) it.next();
     }
@@ -460,6 +507,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kAcc * N);
+  }
+  // add this CTA's histograms of its first groups to the rows' global ones
+  if (use_hist && run) {
+    for (int i = threadIdx.x; i < kHistSlots * NQ * (kHistBins / 2); i += kThreads) {
+      const uint32_t v = S.hist[i];
+      if (v == 0u) continue;
+      const int sq = i / (kHistBins / 2), w = i - sq * (kHistBins / 2);
+      const int row = (g_first + sq / NQ) * NQ + sq % NQ;
+      if (row >= a.num_rows) continue;
+      uint32_t* dst = a.hist + (int64_t)row * kHistBins + 2 * w;
+      if (v & 0xFFFFu) atomicAdd(dst, v & 0xFFFFu);
+      if (v >> 16) atomicAdd(dst + 1, v >> 16);
+    }
   }
 }
 
@@ -507,6 +567,7 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     t.map = a.map;
     t.scores = a.scores + (int64_t)r0 * a.ld_scores;
     t.ld = a.ld_scores;
+    t.hist = a.hist ? a.hist + (int64_t)r0 * kHistBins : nullptr;
     t.status = a.status;
     t.trace = trace_buffer();
     t.spin_limit = fault_spin_limit();
@@ -553,6 +614,10 @@ bool indexer_tc_supported(const IndexerArgs& a) {
   if (a.map.num_tokens >= (int64_t)INT32_MAX) return false;
   if (encode_fn() == nullptr) return false;
   return a.q_group == 1 || a.q_group == 2 || a.q_group == 4;
+}
+
+bool indexer_tc_hist_supported(const IndexerArgs& a) {
+  return indexer_tc_supported(a) && a.q_group <= 2;
 }
 
 size_t indexer_ws_bytes(int num_rows, int q_group) {

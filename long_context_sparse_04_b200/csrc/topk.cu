@@ -58,6 +58,7 @@ struct TopkSmem {
   uint32_t gather[kGatherCap];           // keys of bin B0 of the whole row, by rank
   uint32_t lhist[2][kBins];              // local histograms of the last two digits
   uint32_t above[kMaxCluster];           // keys above bin B0, per rank
+  uint32_t cnt_b0[kMaxCluster];          // keys in bin B0, per rank (fused path)
   uint32_t slice_tot[kMaxCluster];       // slice totals of every CTA
   uint32_t counts[kMaxCluster][2];       // (n_gt, n_eq) of every CTA (radix path)
   uint32_t warp_tmp[kWarps];
@@ -210,6 +211,10 @@ __device__ void cluster_select(TopkSmem& S, int nbins, uint32_t need, uint32_t c
   search_bins(S, S.slice, owner != rank, owner, slice, (int)owner * slice, above, need);
 }
 
+// kHist: the indexer has built each row's histogram of bits 31..20 (a.hist);
+// the first selection pass and its cluster merge are skipped, and the row's
+// histogram is zeroed once every CTA of the row has read it.
+template <bool kHist>
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smraw);
@@ -224,9 +229,12 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const int klen = a.row_klen[t];
   int32_t* out = a.idx + (int64_t)t * k;
 
+  uint32_t* const ghist = kHist ? a.hist + (int64_t)t * kBins0 : nullptr;
   kstamp(a.trace, csize, rank, 0);
   if (klen <= k) {  // uniform over the cluster; no DSMEM was touched
     for (int i = rank * kThreads + tid; i < k; i += csize * kThreads) out[i] = i < klen ? i : -1;
+    if (kHist)
+      for (int i = rank * kThreads + tid; i < kBins0; i += csize * kThreads) ghist[i] = 0u;
     return;
   }
 
@@ -245,7 +253,12 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     for (int i = 4 * n4 + tid; i < ncache; i += kThreads)
       S.keys[i] = __float_as_uint(__ldcg(srow + i));
   }
-  for (int i = tid; i < kBins0; i += kThreads) S.hist[i] = 0;
+  if (kHist) {
+    for (int i = tid; i < kBins0 / 4; i += kThreads)
+      reinterpret_cast<uint4*>(S.hist)[i] = __ldcg(reinterpret_cast<const uint4*>(ghist) + i);
+  } else {
+    for (int i = tid; i < kBins0; i += kThreads) S.hist[i] = 0;
+  }
   cp_async_wait_all();
   __syncthreads();
   kstamp(a.trace, csize, rank, 1);
@@ -275,13 +288,20 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       const uint4 g = key4(v);
       q[0] = g.x; q[1] = g.y; q[2] = g.z; q[3] = g.w;
     }
-    const int nv = nvalid(v);
+    if (!kHist) {
+      const int nv = nvalid(v);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (j < nv) atomicAdd(&S.hist[q[j] >> 20], 1u);
+      for (int j = 0; j < 4; ++j)
+        if (j < nv) atomicAdd(&S.hist[q[j] >> 20], 1u);
+    }
   }
   kstamp(a.trace, csize, rank, 2);
-  cluster_select(S, kBins0, (uint32_t)k, csize, rank);
+  if (kHist) {
+    __syncthreads();                                  // the keys are converted
+    search_bins(S, S.hist, false, 0, kBins0, 0, 0, (uint32_t)k);
+  } else {
+    cluster_select(S, kBins0, (uint32_t)k, csize, rank);
+  }
   const uint32_t B0 = S.sel_bin, need0 = S.sel_need, c0 = S.sel_cnt;
   kstamp(a.trace, csize, rank, 3);
 
@@ -291,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const int nwords = (n + 31) >> 5;                   // <= 512 = kThreads when use_bits
   for (int i = tid; i < 2 * kBins; i += kThreads) (&S.lhist[0][0])[i] = 0;
   if (tid == 0) S.gcount = 0;
+  uint32_t cb_local = 0, ca_local = 0;                // fused path: keys in bin B0 / above it
   if (use_bits) {
     for (int base = warp * 32; base < nvec; base += kThreads) {
       const int v = base + lane;
@@ -300,7 +321,11 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       const int nv = inb ? nvalid(v) : 0;
       uint32_t m = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) m |= (j < nv && (q[j] >> 20) >= B0) ? (1u << j) : 0u;
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t bin = q[j] >> 20;
+        m |= (j < nv && bin >= B0) ? (1u << j) : 0u;
+        if (kHist && j < nv) { cb_local += bin == B0; ca_local += bin > B0; }
+      }
       m <<= 4 * (lane & 7);
       m |= __shfl_xor_sync(0xffffffffu, m, 1);
       m |= __shfl_xor_sync(0xffffffffu, m, 2);
@@ -308,9 +333,41 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       if ((lane & 7) == 0 && inb) S.bits[v >> 3] = m;
     }
   }
+  if (kHist && !use_bits) {
+    for (int v = tid; v < nvec; v += kThreads) {
+      const uint4 g = key4(v);
+      const uint32_t q[4] = {g.x, g.y, g.z, g.w};
+      const int nv = nvalid(v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (j < nv) { cb_local += (q[j] >> 20) == B0; ca_local += (q[j] >> 20) > B0; }
+    }
+  }
   __syncthreads();
   const uint32_t myword = (use_bits && tid < nwords) ? S.bits[tid] : 0u;
   const uint32_t* const mykeys = &S.keys[32 * tid];
+  // fused path: this segment's counts of bin B0 and above it to every CTA of
+  // the row (the staged path reads them from the per-CTA histograms), then
+  // the row's global histogram is cleared for the next call
+  uint32_t goff_h = 0;
+  if (kHist) {
+    const uint32_t cb = block_sum(cb_local, S.warp_tmp);
+    const uint32_t ca = block_sum(ca_local, S.warp_tmp);
+    if (tid < (int)csize) {
+      if ((uint32_t)tid == rank) {
+        S.cnt_b0[rank] = cb;
+        S.above[rank] = ca;
+      } else {
+        st_dsmem_u32(mapa(&S.cnt_b0[rank], (uint32_t)tid), cb);
+        st_dsmem_u32(mapa(&S.above[rank], (uint32_t)tid), ca);
+      }
+    }
+    cluster_sync();                                   // every CTA has read the row's histogram
+    if (rank == 0)
+      for (int i = tid; i < kBins0 / 4; i += kThreads)
+        reinterpret_cast<uint4*>(ghist)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (uint32_t r = 0; r < rank; ++r) goff_h += S.cnt_b0[r];
+  }
   kstamp(a.trace, csize, rank, 4);
 
   // ---- 3. T, `need`, and this CTA's offsets in the cluster-wide order:
@@ -319,20 +376,24 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   const bool gathered = c0 <= (uint32_t)kGatherCap;   // uniform over the cluster
   if (gathered) {
     // where this CTA's bin-B0 keys go in the gathered list: after those of
-    // lower ranks (their histograms still hold their counts of bin B0)
-    if (warp == 0) {
-      uint32_t hb = 0;
-      if (lane < (int)rank) hb = ld_dsmem_u32(mapa(&S.hist[B0], (uint32_t)lane));
-      hb = __reduce_add_sync(0xffffffffu, hb);
-      if (lane == 0) S.goff = hb;
-    }
-    uint32_t ab = 0;                                  // keys of this segment above bin B0
-    for (int b = (int)B0 + 1 + tid; b < kBins0; b += kThreads) ab += S.hist[b];
-    ab = block_sum(ab, S.warp_tmp);                   // also publishes S.goff
-    const uint32_t goff = S.goff;
-    if (tid < (int)csize) {
-      if ((uint32_t)tid == rank) S.above[rank] = ab;
-      else st_dsmem_u32(mapa(&S.above[rank], (uint32_t)tid), ab);
+    // lower ranks (their histograms still hold their counts of bin B0; the
+    // fused path has exchanged the counts above)
+    uint32_t goff = goff_h;
+    if (!kHist) {
+      if (warp == 0) {
+        uint32_t hb = 0;
+        if (lane < (int)rank) hb = ld_dsmem_u32(mapa(&S.hist[B0], (uint32_t)lane));
+        hb = __reduce_add_sync(0xffffffffu, hb);
+        if (lane == 0) S.goff = hb;
+      }
+      uint32_t ab = 0;                                // keys of this segment above bin B0
+      for (int b = (int)B0 + 1 + tid; b < kBins0; b += kThreads) ab += S.hist[b];
+      ab = block_sum(ab, S.warp_tmp);                 // also publishes S.goff
+      goff = S.goff;
+      if (tid < (int)csize) {
+        if ((uint32_t)tid == rank) S.above[rank] = ab;
+        else st_dsmem_u32(mapa(&S.above[rank], (uint32_t)tid), ab);
+      }
     }
     auto send = [&](uint32_t key) {
       const uint32_t slot = goff + atomicAdd(&S.gcount, 1u);
@@ -560,9 +621,10 @@ dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   int csize = 1;
   while (csize < kMaxCluster && (int64_t)csize * kCacheCap < (int64_t)max_klen) csize <<= 1;
   const size_t smem = sizeof(TopkSmem);
-  static std::atomic<bool> attr_done[kMaxDevices] = {};
-  if (dsa_status st = set_smem_limit_once(reinterpret_cast<const void*>(topk_kernel), smem, attr_done))
-    return st;
+  static std::atomic<bool> attr_done[2][kMaxDevices] = {};
+  const void* fn = a.hist ? reinterpret_cast<const void*>(topk_kernel<true>)
+                          : reinterpret_cast<const void*>(topk_kernel<false>);
+  if (dsa_status st = set_smem_limit_once(fn, smem, attr_done[a.hist ? 1 : 0])) return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.num_rows * csize));
   cfg.blockDim = dim3(kThreads);
@@ -577,7 +639,8 @@ dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, topk_kernel, a);
+  cudaError_t e = a.hist ? cudaLaunchKernelEx(&cfg, topk_kernel<true>, a)
+                         : cudaLaunchKernelEx(&cfg, topk_kernel<false>, a);
   if (e != cudaSuccess) {
     set_error("topk launch: %s", cudaGetErrorString(e));
     return DSA_ERR_CUDA;
