@@ -28,6 +28,11 @@ caches by one dsa_cache_append call.  Its metric is appended tokens/s.
 per head, y = W_out u) for the workload's query rows (32 in decode, 65,536 in
 the 64K prefill) with H = 128, d_c = 512, d_v = 128, d_model = 7168: one
 dsa_output_projection call per step.  Its metric is rows/s.
+
+`--op warmup` measures a warm-up step of the indexer on the 8-16K decode batch
+(default): indexer scores, KL to a seeded teacher with its gradient, and the
+backward to q_I, w and k_I (dsa_indexer_scores, dsa_indexer_kl,
+dsa_indexer_backward).  Its metric is query-rows/s.
 """
 from __future__ import annotations
 
@@ -56,7 +61,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=None,
                     help="decode_128k_paged (path default) or prefill_64k (cache_append default)")
-    ap.add_argument("--op", default="path", choices=["path", "cache_append", "output_projection"])
+    ap.add_argument("--op", default="path",
+                    choices=["path", "cache_append", "output_projection", "warmup"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=4, help="oracle rows per CPU-baseline sample")
@@ -882,6 +888,210 @@ def run_out_proj(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- indexer warm-up
+WARMUP_METRIC = "indexer warm-up query-rows/s (scores, KL to the teacher, backward to q_I, w, k_I)"
+WARMUP_UNIT = "query-rows/s"
+
+
+def warmup_teacher(cfg, inp, ld):
+    """Seeded stand-in for the dense-attention teacher of every row: positive
+    weights with some exact zeros, summing to 1 over the row's visible keys."""
+    import numpy as np
+    klen = inp["row_klen"].astype(int)
+    p = np.zeros((len(klen), ld), np.float32)
+    for t, n in enumerate(klen):
+        r = np.random.default_rng([cfg.seed, 90, t])
+        x = r.random(n) ** 3
+        x[r.random(n) < 0.1] = 0.0
+        x[0] = max(x[0], 1e-3)
+        p[t, :n] = x / x.sum()
+    return p
+
+
+def warmup_flops(inp):
+    """Algorithmic FLOPs of the warm-up backward: per visible (row, key) pair the
+    64 x 128 dot products in fp64 (once for dq and dw, once for dk) and the dq
+    and dk contractions in fp32."""
+    pairs = int(inp["row_klen"].astype("int64").sum())
+    h, d = int(inp["h_idx"]), int(inp["d_idx"])
+    return {"fp64": 2 * 2 * h * d * pairs, "fp32": 2 * 2 * h * d * pairs, "pairs": pairs}
+
+
+def run_warmup(args):
+    import numpy as np
+    import torch
+    rank, world, local = dist_info()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from long_context_sparse_04_b200 import build
+    build.build()
+    from long_context_sparse_04_b200 import _native as N
+    from long_context_sparse_04_b200 import inputs as I
+    from long_context_sparse_04_b200.workload import DeviceWorkload, _vp
+
+    cfg = rank_config(I.CONFIGS[args.workload], rank)
+    inp = I.generate(cfg, with_q=False, threads=max(4, min(32, len(os.sched_getaffinity(0)))))
+    wl = DeviceWorkload(inp, device=dev)
+    T, ld = wl.T, wl.ld
+    p = torch.from_numpy(warmup_teacher(cfg, inp, ld)).to(dev)
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    grad = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    loss = torch.empty(T, dtype=torch.float32, device=dev)
+    H_I, d_I = wl.dims.n_idx_heads, wl.dims.d_idx
+    dq = torch.empty((T, H_I, d_I), dtype=torch.float32, device=dev)
+    dw = torch.empty((T, H_I), dtype=torch.float32, device=dev)
+    dk = torch.zeros((int(inp["k_idx"].shape[0]), d_I), dtype=torch.float32, device=dev)
+    n_kl = N.dsa_workspace_size(wl.dims, wl.rows, N.DSA_OP_INDEXER_KL)
+    ws_kl = torch.zeros(n_kl, dtype=torch.uint8, device=dev)
+    n_bw = N.dsa_workspace_size(wl.dims, wl.rows, N.DSA_OP_INDEXER_BACKWARD)
+    ws_bw = torch.zeros(n_bw, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def step():
+        # one warm-up step over the batch: indexer scores, KL + dL/dI, backward
+        wl.indexer(scores)
+        ev[1].record(stream)
+        N.dsa_indexer_kl(wl.rows, _vp(scores), ld, _vp(p), ld, _vp(grad), ld, _vp(loss), _vp(ws_kl),
+                         n_kl, wl.stream)
+        N.dsa_indexer_backward(wl.dims, wl.rows, wl.cache, _vp(wl.q_idx), _vp(wl.q_scale), _vp(wl.w),
+                               _vp(grad), ld, _vp(dq), _vp(dw), _vp(dk), _vp(ws_bw), n_bw, wl.stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    for ws in (ws_kl, ws_bw):
+        st = N.dsa_read_device_status(_vp(ws), wl.stream)
+        assert st == (0, -1), f"device status {st}"
+    assert N.dsa_read_kernel_trace(_vp(ws_bw), wl.stream) & N.DSA_KERNEL_WARMUP
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    t_end = time.perf_counter() + 1.5
+    while time.perf_counter() < t_end:
+        flush.zero_()
+        step()
+        torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ms, ms_bwd = [], []
+    for _ in range(args.steps):
+        flush.zero_()
+        ev[0].record(stream)
+        step()
+        ev[2].record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append(ev[0].elapsed_time(ev[2]))
+        ms_bwd.append(ev[1].elapsed_time(ev[2]))
+    barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(ms), world, dev)
+    value = throughput(world, T, args.steps, total_ms)
+
+    peaks, peak_kind = measured_peaks()
+    fl = warmup_flops(inp)
+    t_bwd = statistics.mean(ms_bwd) / 1e3
+    clock = peaks.get("sm_max_mhz", 1965.0) * 1e6
+    fp64_peak = 148 * 64 * 2 * clock / 1e12
+    roof = {"kernel": "indexer_kl_kernel + indexer_bwd_{dq,reduce,dk}_kernel", "bound": "alu",
+            "achieved": fl["fp64"] / t_bwd / 1e12, "peak": fp64_peak, "unit": "TFLOP/s",
+            "frac": fl["fp64"] / t_bwd / 1e12 / fp64_peak,
+            "peak_source": "derived (148 SMs x 64 fp64 FMA lanes x 2 x max SM clock): the fp64 dot "
+                           "products of the exact ReLU mask dominate",
+            "traffic": None, "algorithmic_per_launch": fl["fp64"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, n = oracle_warmup_rows_per_s(inp, p.cpu().numpy(), 10.0)
+        cpu = {"value": v, "unit": WARMUP_UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"{n} of {T} rows (scores, KL, backward), float64 NumPy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": WARMUP_METRIC, "value": value, "unit": WARMUP_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8e4m3 scores; fp64 mask dots, fp32 gradients", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg) + "; teacher: seeded positive weights per row",
+                       "rows_per_gpu": T, "pairs": fl["pairs"],
+                       "l2": "flushed before every step (256 MiB write, untimed)",
+                       "parallelism": f"{world} independent ranks (weak scaling)"},
+            "stages": {"backward_ms": 1e3 * t_bwd, "scores_ms": statistics.mean(ms) - 1e3 * t_bwd},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": None,
+            "gpu_launches": 5 * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def oracle_warmup_rows_per_s(inp, p, budget_s):
+    """The oracle's warm-up step (scores, KL, backward) on rows of the batch,
+    for about budget_s seconds."""
+    import numpy as np
+    from oracle import dsa_ref as R
+    T = len(inp["row_klen"])
+    t0 = time.perf_counter()
+    n = 0
+    for t in np.linspace(0, T - 1, T).astype(int):
+        klen = int(inp["row_klen"][t])
+        rows = R.physical_rows(int(inp["row_seq"][t]), np.arange(klen), inp["cache"])
+        kd, qd = R.dequant_keys(inp, rows), R.dequant_queries(inp, t)
+        w = np.asarray(inp["w"][t], dtype=np.float32).astype(np.float64)
+        sc = R.indexer_row(qd, w, kd)
+        _, g = R.indexer_kl_row(p[t, :klen].astype(np.float64), sc)
+        R.indexer_backward_row(qd, w, kd, g)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return n / dt, dt, n
+
+
+def run_warmup_reference(args, cfg):
+    from long_context_sparse_04_b200 import inputs as I
+    inp = I.generate(cfg, with_q=False)
+    ld = ((int(inp["row_klen"].max()) + 127) // 128) * 128
+    p = warmup_teacher(cfg, inp, ld)
+    for _ in range(args.warmup):
+        oracle_warmup_rows_per_s(inp, p, 0.0)
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(args.steps):
+        _, _, k = oracle_warmup_rows_per_s(inp, p, 0.0)
+        n += k
+    dt = time.perf_counter() - t0
+    value = n / dt
+    line = {
+        "impl": "reference", "metric": WARMUP_METRIC, "value": value, "unit": WARMUP_UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg) + "; teacher: seeded positive weights per row",
+                   "rows_per_gpu": len(inp["row_klen"]), "pairs": warmup_flops(inp)["pairs"],
+                   "l2": "flushed before every step (256 MiB write, untimed)",
+                   "parallelism": f"{args.gpus} independent ranks (weak scaling)"},
+        "cpu_baseline": {"value": value, "unit": WARMUP_UNIT, "cores": len(os.sched_getaffinity(0)),
+                         "kind": "oracle", "sample": "1 row per step (scores, KL, backward), float64"},
+        "e2e": {"value": value, "unit": WARMUP_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_out_proj_reference(args, cfg):
     from long_context_sparse_04_b200 import inputs as I
     T = cfg.n_rows
@@ -912,8 +1122,16 @@ def run_out_proj_reference(args, cfg):
 def main():
     args = parse()
     if args.workload is None:
-        args.workload = "prefill_64k" if args.op in ("cache_append", "output_projection") \
-            else "decode_128k_paged"
+        args.workload = {"cache_append": "prefill_64k", "output_projection": "prefill_64k",
+                         "warmup": "decode_16k"}.get(args.op, "decode_128k_paged")
+    if args.op == "warmup":
+        if args.impl == "reference":
+            rank, _, _ = dist_info()
+            if rank != 0:
+                return 0
+            from long_context_sparse_04_b200 import inputs as I
+            return run_warmup_reference(args, I.CONFIGS[args.workload])
+        return run_warmup(args)
     if args.op == "output_projection":
         if args.impl == "reference":
             rank, _, _ = dist_info()

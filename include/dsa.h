@@ -139,7 +139,9 @@ typedef enum {
   DSA_OP_SPARSE_MLA = 2,
   DSA_OP_DECODE_STEP = 3,
   DSA_OP_FORWARD = 4,
-  DSA_OP_CACHE_APPEND = 5
+  DSA_OP_CACHE_APPEND = 5,
+  DSA_OP_INDEXER_KL = 6,
+  DSA_OP_INDEXER_BACKWARD = 7
 } dsa_op;
 
 /* Human-readable name of a status code (static storage). */
@@ -182,6 +184,7 @@ dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status
 #define DSA_KERNEL_CACHE_APPEND 0x40u   /* fused FP8 quantise + cache write */
 #define DSA_KERNEL_OUT_PROJ     0x80u   /* tcgen05 output projection GEMM */
 #define DSA_KERNEL_OUT_PROJ_REDUCE 0x100u   /* split-K sum of the W_out product */
+#define DSA_KERNEL_WARMUP       0x200u   /* indexer warm-up: KL and backward kernels */
 
 /* Synchronise `stream`, return the kernel trace of `ws` in *mask_out and clear it. */
 dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_out);
@@ -378,6 +381,47 @@ size_t dsa_output_projection_ws_size(const dsa_proj_dims* dims, int32_t num_rows
 dsa_status dsa_output_projection(const dsa_proj_dims* dims, int32_t num_rows, const void* o,
                                  const void* w_uv, const void* w_out, void* u, void* y,
                                  void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Indexer warm-up ("DeepSeek Sparse Attention DSA Architecture Guide",
+ * section "Training Mechanics: Dense Warm-Up and KL Alignment", Phase 1): the
+ * indexer learns to match the dense attention.  The teacher p_t of query row
+ * t is the dense attention probabilities of the row summed over heads and
+ * normalised over its visible keys (so it sums to 1); the loss is
+ * L^I = sum_t KL(p_t || softmax(I_t)).
+ *
+ * dsa_indexer_kl: for every row t, over s < klen[t],
+ *     loss[t]    = sum_s p[t,s] (log p[t,s] - log softmax(I[t,:])_s)   (0 log 0 = 0)
+ *     grad[t,s]  = softmax(I[t,:])_s - p[t,s]        ( = dL/dI[t,s] )
+ *   scores  [T, ld_scores] fp32, e.g. dsa_indexer_scores' output
+ *   teacher [T, ld_teacher] fp32, p[t,s] >= 0, summing to 1 over s < klen[t]
+ *   grad    [T, ld_grad] fp32 out (entries s >= klen[t] untouched); loss [T] fp32 out
+ * fp32 arithmetic (expf/logf).  ws: the status block
+ * (dsa_workspace_size(..., DSA_OP_INDEXER_KL)).  dims may be NULL. */
+dsa_status dsa_indexer_kl(const dsa_rows* rows, const float* scores, int64_t ld_scores,
+                          const float* teacher, int64_t ld_teacher, float* grad, int64_t ld_grad,
+                          float* loss, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* dsa_indexer_backward: given g = dL/dI (e.g. dsa_indexer_kl's grad), the
+ * gradients of I[t,s] = sum_j w[t,j] ReLU(q[t,j] . k[s]) with respect to the
+ * dequantised operands (e4m3 code times its scale; the FP8 cast is not
+ * differentiated):
+ *     dw[t,j]   = sum_{s<klen[t]} g[t,s] ReLU(q[t,j] . k[s])
+ *     dq[t,j,:] = sum_{s<klen[t]} g[t,s] w[t,j] [q[t,j] . k[s] > 0] k[s]
+ *     dk[s,:]   = sum over the rows t of s's sequence with klen[t] > s of
+ *                 sum_j g[t,s] w[t,j] [q[t,j] . k[s] > 0] q[t,j]
+ *   q_idx, q_scale, w, cache: as dsa_indexer_scores (H_I = 64, d_I = 128)
+ *   grad [T, ld_grad] fp32
+ *   dq [T, H_I, d_I], dw [T, H_I] fp32 out
+ *   dk [num_tokens, d_I] fp32 out, indexed by the key's physical cache row;
+ *      only rows that some query row of the call sees are written
+ * The ReLU mask is decided exactly (the dot product of the e4m3 codes is exact
+ * in fp64), the rest is fp32 with every sum in a fixed order (deterministic).
+ * CUDA-core kernels.  ws: dsa_workspace_size(dims, rows,
+ * DSA_OP_INDEXER_BACKWARD) bytes (status block + per-row partial sums). */
+dsa_status dsa_indexer_backward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                                const void* q_idx, const float* q_scale, const float* w,
+                                const float* grad, int64_t ld_grad, float* dq, float* dw, float* dk,
+                                void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 #ifdef __cplusplus
 }

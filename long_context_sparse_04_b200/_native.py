@@ -16,10 +16,12 @@ DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
 DSA_ALGO_AUTO, DSA_ALGO_SIMT, DSA_ALGO_STAGED = 0, 1, 2
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_DECODE_STEP, DSA_OP_FORWARD = range(5)
 DSA_OP_CACHE_APPEND = 5
+DSA_OP_INDEXER_KL, DSA_OP_INDEXER_BACKWARD = 6, 7
 DSA_KERNEL_INDEXER_SIMT, DSA_KERNEL_INDEXER_TC, DSA_KERNEL_TOPK = 0x01, 0x02, 0x04
 DSA_KERNEL_MLA_SIMT, DSA_KERNEL_MLA_TC, DSA_KERNEL_MLA_COMBINE = 0x08, 0x10, 0x20
 DSA_KERNEL_CACHE_APPEND = 0x40
 DSA_KERNEL_OUT_PROJ, DSA_KERNEL_OUT_PROJ_REDUCE = 0x80, 0x100
+DSA_KERNEL_WARMUP = 0x200
 DSA_FAULT_INDEXER_ACC_RELEASE = 0x1
 
 
@@ -72,6 +74,10 @@ _SIGS = {
                                    ctypes.c_size_t, _P]),
     "dsa_cache_append": (ctypes.c_int, [_P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
+    "dsa_indexer_kl": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, ctypes.c_int64,
+                                      _P, _P, ctypes.c_size_t, _P]),
+    "dsa_indexer_backward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P, _P, _P,
+                                            _P, ctypes.c_size_t, _P]),
     "dsa_output_projection_ws_size": (ctypes.c_size_t, [_P, ctypes.c_int32]),
     "dsa_output_projection": (ctypes.c_int, [_P, ctypes.c_int32, _P, _P, _P, _P, _P, _P,
                                              ctypes.c_size_t, _P]),
@@ -191,3 +197,15 @@ def dsa_output_projection_ws_size(dims, num_rows) -> int:
 def dsa_output_projection(dims, num_rows, o, w_uv, w_out, u, y, ws, ws_bytes, stream, check=True):
     return _call("dsa_output_projection", _ref(dims), num_rows, o, w_uv, w_out, u, y, ws, ws_bytes,
                  stream, check=check)
+
+
+def dsa_indexer_kl(rows, scores, ld_scores, teacher, ld_teacher, grad, ld_grad, loss, ws, ws_bytes,
+                   stream, check=True):
+    return _call("dsa_indexer_kl", _ref(rows), scores, ld_scores, teacher, ld_teacher, grad, ld_grad,
+                 loss, ws, ws_bytes, stream, check=check)
+
+
+def dsa_indexer_backward(dims, rows, cache, q_idx, q_scale, w, grad, ld_grad, dq, dw, dk, ws, ws_bytes,
+                         stream, check=True):
+    return _call("dsa_indexer_backward", _ref(dims), _ref(rows), _ref(cache), q_idx, q_scale, w, grad,
+                 ld_grad, dq, dw, dk, ws, ws_bytes, stream, check=check)

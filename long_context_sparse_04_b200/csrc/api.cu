@@ -67,6 +67,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kForwardChunkRows = 512;
+constexpr int kWarmupChunkKeys = 4096;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t scores_ld(int max_klen) { return ((int64_t)max_klen + 127) / 128 * 128; }
@@ -170,6 +171,7 @@ struct WsPlan {
   size_t idx = 0, idx_bytes = 0;
   size_t mla = 0, mla_bytes = 0;
   size_t hist = 0, hist_bytes = 0;
+  size_t bwd = 0, bwd_bytes = 0;
   size_t total = 0;
   int64_t ld = 0;
   int chunk_rows = 0;
@@ -212,6 +214,11 @@ WsPlan plan(const dsa_dims* d, const dsa_rows* r, dsa_op op) {
     p.hist = off;
     p.hist_bytes = align_up((size_t)rows * 4096 * sizeof(uint32_t));
     off += p.hist_bytes;
+  }
+  if (op == DSA_OP_INDEXER_BACKWARD) {
+    p.bwd = off;
+    p.bwd_bytes = align_up(warmup_ws_bytes(T, r->max_klen, kWarmupChunkKeys));
+    off += p.bwd_bytes;
   }
   p.total = off;
   return p;
@@ -361,8 +368,9 @@ int32_t dsa_version(void) { return 100; }
 
 size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op) {
   if (op == DSA_OP_CACHE_APPEND) return check_dims(dims) == DSA_OK ? kStatusBytes : 0;
+  if (op == DSA_OP_INDEXER_KL) return kStatusBytes;
   if (check_dims(dims) != DSA_OK || check_rows(rows) != DSA_OK) return 0;
-  if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
+  if (op < DSA_OP_INDEXER || op > DSA_OP_INDEXER_BACKWARD || op == DSA_OP_CACHE_APPEND) return 0;
   return plan(dims, rows, op).total;
 }
 
@@ -671,6 +679,74 @@ dsa_status dsa_cache_append(const dsa_dims* dims, const dsa_cache* cache, int32_
   a.num_seqs = cache->num_seqs;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
   return launch_cache_append(a, (cudaStream_t)stream);
+}
+
+dsa_status dsa_indexer_kl(const dsa_rows* rows, const float* scores, int64_t ld_scores,
+                          const float* teacher, int64_t ld_teacher, float* grad, int64_t ld_grad,
+                          float* loss, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_rows(rows))) return st;
+  if ((st = check_ws(ws, ws_bytes, kStatusBytes))) return st;
+  if (rows->num_rows > 0) CHECK_ARG(scores && teacher && grad && loss, "a tensor pointer is NULL");
+  CHECK_ARG(ld_scores >= rows->max_klen && ld_teacher >= rows->max_klen && ld_grad >= rows->max_klen,
+            "leading dimensions must be >= max_klen");
+  WarmupArgs a{};
+  a.num_rows = rows->num_rows;
+  a.row_seq = rows->row_seq;
+  a.row_klen = rows->row_klen;
+  a.scores = scores;
+  a.ld_scores = ld_scores;
+  a.teacher = teacher;
+  a.ld_teacher = ld_teacher;
+  a.grad = grad;
+  a.ld_grad = ld_grad;
+  a.loss = loss;
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  return launch_indexer_kl(a, (cudaStream_t)stream);
+}
+
+dsa_status dsa_indexer_backward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cache* cache,
+                                const void* q_idx, const float* q_scale, const float* w,
+                                const float* grad, int64_t ld_grad, float* dq, float* dw, float* dk,
+                                void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st;
+  if ((st = check_dims(dims)) || (st = check_rows(rows)) ||
+      (st = check_cache(cache, dims, true, false)))
+    return st;
+  if (rows->num_rows > 0) {
+    CHECK_ARG(q_idx && w && grad && dq && dw && dk, "a tensor pointer is NULL");
+    CHECK_ARG(dims->idx_dtype != DSA_FP8_E4M3 || q_scale, "q_scale is NULL for e4m3");
+  }
+  CHECK_ARG(ld_grad >= rows->max_klen, "ld_grad must be >= max_klen");
+  const WsPlan p = plan(dims, rows, DSA_OP_INDEXER_BACKWARD);
+  if ((st = check_ws(ws, ws_bytes, p.total))) return st;
+  WarmupArgs a{};
+  a.num_rows = rows->num_rows;
+  a.row_seq = rows->row_seq;
+  a.row_klen = rows->row_klen;
+  a.n_idx_heads = dims->n_idx_heads;
+  a.d_idx = dims->d_idx;
+  a.idx_dtype = dims->idx_dtype;
+  a.q_idx = q_idx;
+  a.q_scale = dims->idx_dtype == DSA_FP8_E4M3 ? q_scale : nullptr;
+  a.w = w;
+  a.idx_k = cache->idx_k;
+  a.idx_k_scale = dims->idx_dtype == DSA_FP8_E4M3 ? cache->idx_k_scale : nullptr;
+  a.map = make_map(cache);
+  a.grad = const_cast<float*>(grad);
+  a.ld_grad = ld_grad;
+  a.dq = dq;
+  a.dw = dw;
+  a.dk = dk;
+  a.partial = reinterpret_cast<float*>(at(ws, p.bwd));
+  a.chunk_keys = kWarmupChunkKeys;
+  a.n_chunks = (rows->max_klen + kWarmupChunkKeys - 1) / kWarmupChunkKeys;
+  a.status = reinterpret_cast<DeviceStatus*>(ws);
+  if (!warmup_supported(a)) {
+    set_error("indexer backward runs H_I = 64, d_I = 128 (e4m3 or f32)");
+    return DSA_ERR_UNSUPPORTED;
+  }
+  return launch_indexer_backward(a, rows->max_klen, cache->num_seqs, (cudaStream_t)stream);
 }
 
 size_t dsa_output_projection_ws_size(const dsa_proj_dims* dims, int32_t num_rows) {

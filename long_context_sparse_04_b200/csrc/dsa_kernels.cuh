@@ -107,6 +107,39 @@ size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
 dsa_status launch_cache_append(const AppendArgs& a, cudaStream_t stream);
 int cache_append_max_d_idx();
 
+// Indexer warm-up: KL(p || softmax(I)) per row, its gradient g, and the
+// backward of the indexer scores to q_I, w and k_I.
+struct WarmupArgs {
+  int num_rows;
+  const int32_t* row_seq;
+  const int32_t* row_klen;
+  int n_idx_heads, d_idx;
+  dsa_dtype idx_dtype;
+  const void* q_idx;          // [T, H_I, d_I]
+  const float* q_scale;       // [T, H_I] or null
+  const float* w;             // [T, H_I]
+  const void* idx_k;          // [num_tokens, d_I]
+  const float* idx_k_scale;   // [num_tokens] or null
+  CacheMap map;
+  const float* scores;        // KL: [T, ld_scores]
+  int64_t ld_scores;
+  const float* teacher;       // KL: [T, ld_teacher]
+  int64_t ld_teacher;
+  float* grad;                // KL: written; backward: read.  [T, ld_grad]
+  int64_t ld_grad;
+  float* loss;                // KL: [T]
+  float* dq;                  // backward: [T, H_I, d_I]
+  float* dw;                  // backward: [T, H_I]
+  float* dk;                  // backward: [num_tokens, d_I] (rows some query sees)
+  float* partial;             // backward workspace: [T, n_chunks, H_I, d_I + 1]
+  int chunk_keys, n_chunks;
+  DeviceStatus* status;
+};
+bool warmup_supported(const WarmupArgs& a);
+size_t warmup_ws_bytes(int num_rows, int max_klen, int chunk_keys);
+dsa_status launch_indexer_kl(const WarmupArgs& a, cudaStream_t stream);
+dsa_status launch_indexer_backward(const WarmupArgs& a, int max_klen, int num_seqs, cudaStream_t stream);
+
 // Output projection: u = W_UV,i o_i per head, then y = W_out [u_1; ...; u_H].
 struct ProjArgs {
   int num_rows, n_heads, d_c, d_v, d_model;

@@ -16,13 +16,14 @@
 // physical cache row of both 64-key halves of every tile of the range into
 // shared memory, so the loops below never wait on a dependent global load.
 // Roles (576 threads):
-//   warp 0      producer: one thread issues the TMA of the two 64-row key
-//               boxes (a box never crosses a 64-token page) into a 10-stage
-//               ring (6 when N = 256), and of the group's queries (N x 128 B)
-//               into a double buffer; the 32 lanes copy the tile's 128 key
-//               scales into a scale slot with cp.async, so the epilogue never
-//               waits on a global load.  Per-tile flags computed in the
-//               prologue (first / last tile of its group) keep this loop short.
+//   warp 0      producer (one thread): TMA of the two 64-row key boxes (a box
+//               never crosses a 64-token page) into an 8-stage ring (6 when
+//               N = 256), and of the group's queries (N x 128 B) into a double
+//               buffer.  Per-tile flags computed in the prologue (first / last
+//               tile of its group) keep this loop short.
+//   warp 18     key scales: the 32 lanes copy each tile's 128 key scales into
+//               a scale slot with cp.async, a stage at a time behind the
+//               producer, so the epilogue never waits on a global load.
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (kind::f8f6f4, e4m3 x e4m3 -> fp32, 4 MMAs of K=32 per tile)
 //               into one of four (N <= 128) or two TMEM accumulators; one
@@ -46,7 +47,8 @@ constexpr int kTileKeys = 128;
 constexpr int kDI = 128;
 constexpr int kHI = 64;
 constexpr int kEpiWarps = 16;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kScaleWarp = 2 + kEpiWarps;          // warp 18: key scales into their slots
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32;
 constexpr int kMaxGroups = 2048;
 // At most 511 tiles per CTA: a row's key count inside one CTA then stays below
 // 65,536, so the shared-memory score histogram can keep 16-bit counters.
@@ -290,88 +292,54 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   }
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Lane 0 issues the TMA loads of the keys (and of the queries); every lane
-    // then copies 4 of the tile's 128 key scales into the scale slot with
-    // cp.async, whose completion also arrives on the stage's full barrier.
-    if (run) {
-      // A lean loop: one thread issues every bulk load, so its instruction
-      // count per tile bounds the tile rate.
-      if (lane == 0) {
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_q);
-      }
-      const bool tracing = a.trace != nullptr && blockIdx.x == 0 && lane == 0;
-      const int half = lane >> 4, k4 = 4 * (lane & 15);
+    // ------------------------------------------------------------ producer (lane 0): TMA only
+    if (run && lane == 0) {
+      // A lean loop: one thread issues every load, so its instruction count
+      // per tile bounds the tile rate.
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_q);
+      const bool tracing = a.trace != nullptr && blockIdx.x == 0;
       int st = 0, qb = 0;
       uint32_t ph = 1, qph = 1;                       // parity to wait for on empty / q_empty
-      int qcount = 0, j = 0;
+      int qcount = 0, qloads = 0, j = 0;
       bool alive = true;
       for (; j < ntile; ++j) {
         const int info = S.tile_info[j];
         const int2 rr = *reinterpret_cast<const int2*>(S.tile_row[j]);
-        if (lane == 0) {
-          if (info & 1) {
-            if (qcount > 0) { qb ^= 1; if (qb == 0) qph ^= 1; }
-            ++qcount;
-            alive = mbar_wait(&S.q_empty[qb], qph, a.status, 1, lim);
-            if (alive) {
-              mbar_expect_tx(&S.q_full[qb], kQBytes);
-              tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, (info >> 2) * NQ * kHI);
-            }
-          }
-          alive = alive && mbar_wait(&S.empty[st], ph, a.status, 2, lim);
+        if (info & 1) {
+          if (qcount > 0) { qb ^= 1; if (qb == 0) qph ^= 1; }
+          ++qcount;
+          if (!(alive = mbar_wait(&S.q_empty[qb], qph, a.status, 1, lim))) break;
+          mbar_expect_tx(&S.q_full[qb], kQBytes);
+          tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, (info >> 2) * NQ * kHI);
+          ++qloads;
         }
-        alive = __shfl_sync(0xffffffffu, alive, 0);   // uniform: the stage is free
-        if (!alive) break;
-        if (lane == 0) {
-          if (tracing) istamp(a.trace, 0, j);
-          const uint32_t bytes = (rr.x >= 0 ? kKeyTileBytes / 2 : 0) + (rr.y >= 0 ? kKeyTileBytes / 2 : 0);
-          if (bytes == 0) {
-            mbar_arrive(&S.full[st]);
-          } else {
-            mbar_expect_tx(&S.full[st], bytes);
-            if (rr.x >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, rr.x);
-            if (rr.y >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, rr.y);
-          }
-          if (tracing) istamp(a.trace, 1, j);
+        if (!(alive = mbar_wait(&S.empty[st], ph, a.status, 2, lim))) break;
+        if (tracing) istamp(a.trace, 0, j);
+        const uint32_t bytes = (rr.x >= 0 ? kKeyTileBytes / 2 : 0) + (rr.y >= 0 ? kKeyTileBytes / 2 : 0);
+        if (bytes == 0) {
+          mbar_arrive(&S.full[st]);
+        } else {
+          mbar_expect_tx(&S.full[st], bytes);
+          if (rr.x >= 0) tma_load_2d(S.keys[st], &tm_k, &S.full[st], 0, rr.x);
+          if (rr.y >= 0) tma_load_2d(S.keys[st] + kKeyTileBytes / 2, &tm_k, &S.full[st], 0, rr.y);
         }
-        // scales of keys [64 half + k4, +4): one 16-byte piece when aligned and in
-        // range, else four 4-byte pieces (rows past the cache read as 0)
-        {
-          const int row = half ? rr.y : rr.x;
-          float* dst = &S.kscale[j % kScaleSlots][64 * half + k4];
-          const int64_t pr = (int64_t)row + k4;
-          if (row >= 0 && (reinterpret_cast<uintptr_t>(a.k_scale + pr) & 15) == 0 &&
-              pr + 4 <= a.map.num_tokens) {
-            cp_async_16(dst, a.k_scale + pr);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const bool ok = row >= 0 && pr + e < a.map.num_tokens;
-              cp_async_4_zfill(dst + e, a.k_scale + (ok ? pr + e : 0), ok);
-            }
-          }
-          cp_async_mbar_arrive(&S.full[st]);
-        }
+        if (tracing) istamp(a.trace, 1, j);
         if (++st == kStages) { st = 0; ph ^= 1; }
       }
-      cp_async_wait_all();
       // tail: every bulk load issued has landed (also when a wait above ran
       // out and the MMA stopped consuming), then the MMAs have released every
       // stage and query buffer in use, so nothing is still in flight to this
       // CTA's shared memory at exit
-      if (lane == 0) {
-        for (int s2 = 0; s2 < kStages && s2 < j; ++s2) {
-          const int fills = (j - 1 - s2) / kStages + 1;
-          if (!mbar_wait(&S.full[s2], (fills - 1) & 1, a.status, 9, lim)) break;
-        }
-        for (int q2 = 0; q2 < 2 && q2 < qcount; ++q2) {
-          const int fills = (qcount - q2 + 1) / 2;
-          if (!mbar_wait(&S.q_full[q2], (fills - 1) & 1, a.status, 10, lim)) break;
-        }
+      for (int s2 = 0; s2 < kStages && s2 < j; ++s2) {
+        const int fills = (j - 1 - s2) / kStages + 1;
+        if (!mbar_wait(&S.full[s2], (fills - 1) & 1, a.status, 9, lim)) break;
       }
-      if (alive && lane == 0) {
+      for (int q2 = 0; q2 < 2 && q2 < qloads; ++q2) {
+        const int fills = (qloads - q2 + 1) / 2;
+        if (!mbar_wait(&S.q_full[q2], (fills - 1) & 1, a.status, 10, lim)) break;
+      }
+      if (alive) {
         for (int s2 = 0; s2 < kStages && s2 < j; ++s2) {
           const int last_use = (j - 1 - s2) / kStages;
           if (!mbar_wait(&S.empty[s2], last_use & 1, a.status, 7, lim)) break;
@@ -381,6 +349,42 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           if (!mbar_wait(&S.q_empty[q2], last_use & 1, a.status, 8, lim)) break;
         }
       }
+    }
+  } else if (warp == kScaleWarp) {
+    // ------------------------------------------------------------ key scales (32 lanes)
+    // Follows the producer stage by stage: once a stage is free (the same
+    // wait as the producer's), each lane copies 4 of the tile's 128 key
+    // scales into the tile's scale slot with cp.async, whose completion
+    // arrives on the stage's full barrier.  A separate warp keeps this work
+    // out of the producer's loop.
+    if (run) {
+      const int half = lane >> 4, k4 = 4 * (lane & 15);
+      int st = 0;
+      uint32_t ph = 1;
+      for (int j = 0; j < ntile; ++j) {
+        const int2 rr = *reinterpret_cast<const int2*>(S.tile_row[j]);
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&S.empty[st], ph, a.status, 11, lim);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        // scales of keys [64 half + k4, +4): one 16-byte piece when aligned and
+        // in range, else four 4-byte pieces (rows past the cache read as 0)
+        const int row = half ? rr.y : rr.x;
+        float* dst = &S.kscale[j % kScaleSlots][64 * half + k4];
+        const int64_t pr = (int64_t)row + k4;
+        if (row >= 0 && (reinterpret_cast<uintptr_t>(a.k_scale + pr) & 15) == 0 &&
+            pr + 4 <= a.map.num_tokens) {
+          cp_async_16(dst, a.k_scale + pr);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool in = row >= 0 && pr + e < a.map.num_tokens;
+            cp_async_4_zfill(dst + e, a.k_scale + (in ? pr + e : 0), in);
+          }
+        }
+        cp_async_mbar_arrive(&S.full[st]);
+        if (++st == kStages) { st = 0; ph ^= 1; }
+      }
+      cp_async_wait_all();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -418,7 +422,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       }
     }
   } else if (run) {
-    // ------------------------------------------------------------ epilogue (16 warps)
+    // ------------------------------------------------------------ epilogue (warps 2-17)
     // The 16 warps form NSET = 16 / (4*NQ) sets of 4*NQ warps; set k takes the
     // tiles j = k (mod NSET), so the sets sit in different phases and one set's
     // TMEM-load latency overlaps another's arithmetic.  Warp (lq, qi) of a set
@@ -461,6 +465,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       tmem_ld32(col + 32, v1);
       tmem_wait_ld_regs(v0);
       tmem_wait_ld_regs(v1);
+      if (threadIdx.x == 64) istamp(a.trace, 6, j);
       tc_fence_before();
       __syncwarp();
       // values are in registers (a test may withhold the release, so that the

@@ -470,13 +470,17 @@ def indexer_kl_row(p: np.ndarray, scores: np.ndarray):
     return kl, np.exp(log_q) - p
 
 
-def indexer_backward_row(q: np.ndarray, w: np.ndarray, k: np.ndarray, g: np.ndarray):
+def indexer_backward_row(q: np.ndarray, w: np.ndarray, k: np.ndarray, g: np.ndarray, on=None):
     """Backward of I[s] = sum_j w[j] ReLU(q[j] . k[s]) for one row, given
     g[s] = dL/dI[s].  q [H_I, d_I], w [H_I], k [n, d_I], g [n].  ReLU's
     derivative is 1 where its argument is > 0 and 0 elsewhere (0 at 0).
+    `on` [n, H_I] (optional) gives that decision, [q[j] . k[s] > 0], taken
+    exactly elsewhere (for FP8 operands: the sign of the dot product of the
+    codes, as the scales are positive); by default it is taken from the
+    float64 dot products here.
     Returns (dq [H_I, d_I], dw [H_I], dk [n, d_I])."""
     d = k @ q.T                               # [n, H_I]
-    on = (d > 0).astype(np.float64)
+    on = (d > 0).astype(np.float64) if on is None else np.asarray(on, dtype=np.float64)
     dw = np.maximum(d, 0.0).T @ g             # [H_I]
     gd = (g[:, None] * on) * w[None, :]       # dL/d(q_j . k_s), [n, H_I]
     dq = gd.T @ k                             # [H_I, d_I]

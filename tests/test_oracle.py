@@ -558,3 +558,27 @@ def test_indexer_backward_against_autograd():
     np.testing.assert_allclose(dq_o, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dw_o, tw.grad.numpy(), rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dk_o, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_mask_argument_is_the_relu_decision():
+    # passing the ReLU decision explicitly changes nothing when it is the one
+    # the float64 dot products give; for FP8 operands the exact decision (the
+    # sign of the codes' dot product, scales being positive) agrees with them
+    # except where the float64 dot product is within rounding of zero
+    rng = np.random.default_rng(26)
+    q, w, k = rng.standard_normal((4, 6)), rng.standard_normal(4), rng.standard_normal((9, 6))
+    g = rng.standard_normal(9)
+    a = R.indexer_backward_row(q, w, k, g)
+    b = R.indexer_backward_row(q, w, k, g, on=(k @ q.T) > 0)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    codes_q = rng.integers(0, 256, (64, 128)).astype(np.uint8)
+    codes_k = rng.integers(0, 256, (50, 128)).astype(np.uint8)
+    codes_q[(codes_q & 0x7F) == 0x7F] = 0                       # no NaN codes
+    codes_k[(codes_k & 0x7F) == 0x7F] = 0
+    qs, ks = rng.random(64) + 0.5, rng.random(50) + 0.5
+    qc, kc = R.e4m3_decode(codes_q), R.e4m3_decode(codes_k)
+    exact = (kc @ qc.T) > 0
+    d = (kc * ks[:, None]) @ (qc * qs[:, None]).T
+    near = np.abs(d) <= 1e-12 * (np.abs(kc * ks[:, None]) @ np.abs(qc * qs[:, None]).T)
+    assert np.array_equal(exact[~near], (d > 0)[~near])

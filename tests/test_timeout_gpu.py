@@ -15,8 +15,8 @@ from tests import parity as P
 pytestmark = pytest.mark.gpu
 
 # wait sites of the indexer kernel: producer (1, 2), MMA issuer (3, 4, 5),
-# epilogue (6), producer tail (7, 8, 9, 10)
-INDEXER_SITES = set(range(1, 11))
+# epilogue (6), producer tail (7, 8, 9, 10), key-scale warp (11)
+INDEXER_SITES = set(range(1, 12))
 
 
 @pytest.fixture(scope="module")
