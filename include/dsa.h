@@ -196,12 +196,18 @@ dsa_status dsa_read_kernel_trace(void* ws, dsa_stream_t stream, uint32_t* mask_o
  * n_events = 0 turns this off.  The handles are not owned by the library. */
 dsa_status dsa_set_stage_events(void* const* events, int32_t n_events);
 
-/* Profiling trace on the calling thread.  When `dev_buf` (device memory,
- * `bytes` long, zeroed by the caller) is set, the sparse-MLA kernel's first CTA
- * pair records clock64() stamps of its pipeline events there: int64
- * [2 CTAs][8 events][32 blocks] (gather issued, gather landed, S issued, PV
- * issued, logits ready, exchange done, P stored, exchange slot free).
- * dev_buf = NULL turns it off.  For performance analysis only. */
+/* Profiling trace on the calling thread.  When `dev_buf` (device memory, at
+ * least 896 int64 = 7168 bytes, zeroed by the caller) is set, the tensor-core
+ * kernels record clock64() stamps of their pipeline events there, each in its
+ * own region: int64 [0, 512) the sparse-MLA kernel's first CTA pair
+ * ([2 CTAs][8 events][32 blocks]: decoded, after the max barrier, S issued,
+ * PV issued, S read by the softmax, peer logits arrived, P stored, exp done),
+ * [512, 640) top-k's first cluster ([8 CTAs][16 events], phase ends), and
+ * [640, 896) the indexer's CTA 0 ([8 events][32 tiles]: stage free, TMA
+ * issued, MMA ready, MMA committed, accumulator ready, key data landed,
+ * accumulator loaded, scores stored).  Stamps of one SM's clock; compare
+ * within a region.  dev_buf = NULL turns it off.  For performance analysis
+ * only. */
 dsa_status dsa_set_trace_buffer(void* dev_buf, size_t bytes);
 
 /* Fault injection, for tests of the failure paths only (never set it in

@@ -300,7 +300,7 @@ MlaArgs mla_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c, const
   a.splits = p.splits;
   a.part_o = reinterpret_cast<float*>(at(ws, p.mla));
   a.part_ml = a.part_o + (size_t)r->num_rows * p.splits * d->n_heads * d->d_c;
-  a.trace = trace_buffer();
+  a.trace = trace_buffer() ? trace_buffer() + kTraceMla : nullptr;
   return a;
 }
 
@@ -436,8 +436,8 @@ dsa_status dsa_set_stage_events(void* const* events, int32_t n_events) {
 }
 
 dsa_status dsa_set_trace_buffer(void* dev_buf, size_t bytes) {
-  if (dev_buf != nullptr && bytes < sizeof(long long) * 2 * kTraceEvents * kTraceBlocks) {
-    set_error("trace buffer needs %zu bytes", sizeof(long long) * 2 * kTraceEvents * kTraceBlocks);
+  if (dev_buf != nullptr && bytes < sizeof(long long) * kTraceLen) {
+    set_error("trace buffer needs %zu bytes", sizeof(long long) * kTraceLen);
     return DSA_ERR_INVALID_ARG;
   }
   g_trace = static_cast<long long*>(dev_buf);
@@ -496,7 +496,7 @@ dsa_status dsa_topk(const dsa_dims* dims, const dsa_rows* rows, const float* sco
   a.topk = dims->topk;
   a.idx = idx;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
-  a.trace = trace_buffer();
+  a.trace = trace_buffer() ? trace_buffer() + kTraceTopk : nullptr;
   return launch_topk(a, rows->max_klen, (cudaStream_t)stream);
 }
 
@@ -577,7 +577,7 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   ta.topk = dims->topk;
   ta.idx = idx;
   ta.status = reinterpret_cast<DeviceStatus*>(ws);
-  ta.trace = trace_buffer();
+  ta.trace = trace_buffer() ? trace_buffer() + kTraceTopk : nullptr;
   ta.hist = ia.hist;
   if ((st = launch_topk(ta, rows->max_klen, s))) return st;
   stage_event(2, s);
@@ -635,7 +635,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     ta.topk = dims->topk;
     ta.idx = idx;
     ta.status = reinterpret_cast<DeviceStatus*>(ws);
-    ta.trace = trace_buffer();
+    ta.trace = trace_buffer() ? trace_buffer() + kTraceTopk : nullptr;
     ta.hist = ia.hist;
     if ((st = launch_topk(ta, rows->max_klen, s))) return st;
     MlaArgs ma = mla_args(dims, &cr, cache, qq, idx, oo, ll, ws, p);

@@ -79,7 +79,11 @@ struct AppendArgs {
 };
 
 // Profiling trace buffer registered on the calling host thread (or null).
+// Layout (int64 clock64 stamps): [0, 512) the attention kernel's first CTA
+// pair ([2 CTAs][8 events][32 blocks]), [512, 640) top-k's first cluster
+// ([8 CTAs][16 events]), [640, 896) the indexer's CTA 0 ([8 events][32 tiles]).
 long long* trace_buffer();
+constexpr int kTraceMla = 0, kTraceTopk = 512, kTraceIdx = 640, kTraceLen = 896;
 // Test-only fault injection of the calling host thread (dsa_set_fault_injection):
 // the spin limit of the kernels' bounded waits (kSpinLimit unless set) and the
 // DSA_FAULT_* bits to inject.

@@ -574,7 +574,7 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     t.ld = a.ld_scores;
     t.hist = a.hist ? a.hist + (int64_t)r0 * kHistBins : nullptr;
     t.status = a.status;
-    t.trace = trace_buffer();
+    t.trace = trace_buffer() ? trace_buffer() + kTraceIdx : nullptr;
     t.spin_limit = fault_spin_limit();
     t.inject = fault_inject();
     CUtensorMap tq;

@@ -254,14 +254,18 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       S.keys[i] = __float_as_uint(__ldcg(srow + i));
   }
   if (kHist) {
+    // the threshold bin from the row's histogram, while the segment lands
     for (int i = tid; i < kBins0 / 4; i += kThreads)
       reinterpret_cast<uint4*>(S.hist)[i] = __ldcg(reinterpret_cast<const uint4*>(ghist) + i);
+    __syncthreads();
+    search_bins(S, S.hist, false, 0, kBins0, 0, 0, (uint32_t)k);
   } else {
     for (int i = tid; i < kBins0; i += kThreads) S.hist[i] = 0;
   }
   cp_async_wait_all();
   __syncthreads();
   kstamp(a.trace, csize, rank, 1);
+  const bool use_bits = n <= kCacheCap;               // uniform over the CTA
 
   // four keys starting at 4v (converted); entries at or past n are garbage
   auto key4 = [&](int v) -> uint4 {
@@ -274,8 +278,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   auto nvalid = [&](int v) { return min(4, n - 4 * v); };
 
   // ---- 1. keys in place, histogram of bits 31..20, cluster-wide bin B0
+  // (the fused path converts the keys in the bitmap pass below)
 #pragma unroll 2
-  for (int v = tid; v < nvec; v += kThreads) {
+  for (int v = tid; v < ((kHist && use_bits) ? 0 : nvec); v += kThreads) {
     uint32_t q[4];
     if (4 * v < ncache) {
       const uint4 raw = *reinterpret_cast<const uint4*>(&S.keys[4 * v]);
@@ -296,18 +301,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     }
   }
   kstamp(a.trace, csize, rank, 2);
-  if (kHist) {
-    __syncthreads();                                  // the keys are converted
-    search_bins(S, S.hist, false, 0, kBins0, 0, 0, (uint32_t)k);
-  } else {
-    cluster_select(S, kBins0, (uint32_t)k, csize, rank);
-  }
+  if (!kHist) cluster_select(S, kBins0, (uint32_t)k, csize, rank);
   const uint32_t B0 = S.sel_bin, need0 = S.sel_need, c0 = S.sel_cnt;
   kstamp(a.trace, csize, rank, 3);
 
   // ---- 2. bitmap of the keys in bin B0 or above (segments held in smem):
-  // lanes 8i..8i+7 of a round hold the 32 keys of one word
-  const bool use_bits = n <= kCacheCap;               // uniform over the CTA
+  // lanes 8i..8i+7 of a round hold the 32 keys of one word; the fused path
+  // turns the scores into keys here, in the same pass (thread tid holds the
+  // same vectors tid, tid + 512, ... as the conversion loop above)
   const int nwords = (n + 31) >> 5;                   // <= 512 = kThreads when use_bits
   for (int i = tid; i < 2 * kBins; i += kThreads) (&S.lhist[0][0])[i] = 0;
   if (tid == 0) S.gcount = 0;
@@ -316,7 +317,12 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     for (int base = warp * 32; base < nvec; base += kThreads) {
       const int v = base + lane;
       const bool inb = v < nvec;
-      const uint4 g = inb ? *reinterpret_cast<const uint4*>(&S.keys[4 * v]) : make_uint4(0, 0, 0, 0);
+      uint4 g = inb ? *reinterpret_cast<const uint4*>(&S.keys[4 * v]) : make_uint4(0, 0, 0, 0);
+      if (kHist && inb) {
+        g = make_uint4(float_key(__uint_as_float(g.x)), float_key(__uint_as_float(g.y)),
+                       float_key(__uint_as_float(g.z)), float_key(__uint_as_float(g.w)));
+        *reinterpret_cast<uint4*>(&S.keys[4 * v]) = g;
+      }
       const uint32_t q[4] = {g.x, g.y, g.z, g.w};
       const int nv = inb ? nvalid(v) : 0;
       uint32_t m = 0;
@@ -351,8 +357,15 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   // the row's global histogram is cleared for the next call
   uint32_t goff_h = 0;
   if (kHist) {
-    const uint32_t cb = block_sum(cb_local, S.warp_tmp);
-    const uint32_t ca = block_sum(ca_local, S.warp_tmp);
+    uint32_t cb, ca;
+    if (use_bits) {                                   // both counts <= 16384: one packed sum
+      const uint32_t both = block_sum((ca_local << 16) | cb_local, S.warp_tmp);
+      cb = both & 0xFFFFu;
+      ca = both >> 16;
+    } else {
+      cb = block_sum(cb_local, S.warp_tmp);
+      ca = block_sum(ca_local, S.warp_tmp);
+    }
     if (tid < (int)csize) {
       if ((uint32_t)tid == rank) {
         S.cnt_b0[rank] = cb;
