@@ -67,7 +67,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kForwardChunkRows = 512;
-constexpr int kWarmupChunkKeys = 4096;
+constexpr int kWarmupChunkKeys = 512;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 int64_t scores_ld(int max_klen) { return ((int64_t)max_klen + 127) / 128 * 128; }

@@ -129,18 +129,29 @@ __device__ __forceinline__ void load_query(const WarmupArgs& a, int t, float (*q
 }
 
 // dots[s][j] = sum_i kv[s][i] qv[j][i] in fp64 (exact for e4m3 values), for
-// the 32 x 64 (key, head) pairs of a tile: 8 per thread.
+// the 32 x 64 (key, head) pairs of a tile.  Thread tid takes keys ks, ks + 16
+// (ks = tid / 16) and heads jh + 16c (jh = tid % 16, c < 4): 6 shared loads per
+// 8 FMAs.  Each thread walks the dims from its own start 2 jh + ks, so the 32
+// lanes of a warp read 32 different banks.
 __device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kDI], double (*dots)[kHI]) {
-#pragma unroll 1
-  for (int e = threadIdx.x; e < kTile * kHI; e += kThreads) {
-    const int s = e / kHI, j = e - s * kHI;
-    double acc = 0.0;
-#pragma unroll 8
-    for (int i = 0; i < kDI; ++i) {
-      const int ii = (i + j) & (kDI - 1);              // rotated start: fewer bank conflicts
-      acc = fma((double)kv[s][ii], (double)qv[j][ii], acc);
+  const int ks = threadIdx.x >> 4, jh = threadIdx.x & 15;
+  const int rot = 2 * jh + ks;
+  double acc[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
+#pragma unroll 4
+  for (int i = 0; i < kDI; ++i) {
+    const int ii = (i + rot) & (kDI - 1);
+    const double k0 = kv[ks][ii], k1 = kv[ks + 16][ii];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const double q = qv[jh + 16 * c][ii];
+      acc[0][c] = fma(k0, q, acc[0][c]);
+      acc[1][c] = fma(k1, q, acc[1][c]);
     }
-    dots[s][j] = acc;
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    dots[ks][jh + 16 * c] = acc[0][c];
+    dots[ks + 16][jh + 16 * c] = acc[1][c];
   }
   __syncthreads();
 }
@@ -155,7 +166,7 @@ struct DqSmem {
 };
 
 // grid (n_chunks, T), block 256.  Thread tid accumulates dq[j][d] for
-// j = tid / 4 (heads 0..63) and d = 32 (tid % 4) + 0..31, and (tid < 64) dw[tid].
+// j = tid / 4 (heads 0..63) and d = tid % 4 + 4i (i < 32), and (tid < 64) dw[tid].
 __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   DqSmem& S = *reinterpret_cast<DqSmem*>(smraw);
@@ -163,7 +174,7 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) 
   const int t = blockIdx.y, c = blockIdx.x;
   const int klen = a.row_klen[t], seq = a.row_seq[t];
   const int s_lo = c * a.chunk_keys, s_hi = min(klen, s_lo + a.chunk_keys);
-  const int jq = threadIdx.x >> 2, d0 = 32 * (threadIdx.x & 3);
+  const int jq = threadIdx.x >> 2, d0 = threadIdx.x & 3;
   float acc[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) acc[i] = 0.f;
@@ -188,7 +199,7 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) 
       for (int s = 0; s < kTile; ++s) {               // dq_j += sum_s coef_sj k_s
         const float cf = S.coef[s][jq];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = fmaf(cf, S.kv[s][d0 + i], acc[i]);
+        for (int i = 0; i < 32; ++i) acc[i] = fmaf(cf, S.kv[s][d0 + 4 * i], acc[i]);
       }
       __syncthreads();
     }
@@ -196,7 +207,7 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) 
   // partials [T][n_chunks][64][128 + 1]: dq then dw at column 128
   float* part = a.partial + (((int64_t)t * a.n_chunks + c) * kHI) * (kDI + 1);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) part[(int64_t)jq * (kDI + 1) + d0 + i] = acc[i];
+  for (int i = 0; i < 32; ++i) part[(int64_t)jq * (kDI + 1) + d0 + 4 * i] = acc[i];
   if (threadIdx.x < kHI) part[(int64_t)threadIdx.x * (kDI + 1) + kDI] = dw;
 }
 
@@ -224,14 +235,14 @@ struct DkSmem {
 };
 
 // grid (ceil(max_klen / 32), num_seqs), block 256.  Thread tid accumulates
-// dk[s][d] for s = tid / 8 and d = 16 (tid % 8) + 0..15, over the rows of
+// dk[s][d] for s = tid / 8 and d = tid % 8 + 8i (i < 16), over the rows of
 // sequence b that see key s, in row order; writes the keys some row sees.
 __global__ void __launch_bounds__(kThreads) indexer_bwd_dk_kernel(WarmupArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   DkSmem& S = *reinterpret_cast<DkSmem*>(smraw);
   trace_kernel(a.status, DSA_KERNEL_WARMUP);
   const int b = blockIdx.y, s0 = blockIdx.x * kTile;
-  const int sk = threadIdx.x >> 3, d0 = 16 * (threadIdx.x & 7);
+  const int sk = threadIdx.x >> 3, d0 = threadIdx.x & 7;
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
@@ -269,14 +280,14 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dk_kernel(WarmupArgs a) 
     for (int j = 0; j < kHI; ++j) {                   // dk_s += sum_j coef_sj q_j
       const float cf = S.coef[sk][j];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = fmaf(cf, S.qv[j][d0 + i], acc[i]);
+      for (int i = 0; i < 16; ++i) acc[i] = fmaf(cf, S.qv[j][d0 + 8 * i], acc[i]);
     }
     __syncthreads();
   }
   if (S.seen[sk] && S.prow[sk] >= 0) {
     float* dst = a.dk + S.prow[sk] * kDI + d0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) dst[i] = acc[i];
+    for (int i = 0; i < 16; ++i) dst[8 * i] = acc[i];
   }
 }
 
