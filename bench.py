@@ -475,10 +475,11 @@ def measure_path(args, cfg, dev, rank: int, world: int, steps: int, warmup: int,
 
 
 def path_launches(N, ran: int, T: int, prefill: bool) -> int:
-    """Kernels of this library one step launches."""
-    if prefill:   # three kernels per 512-row chunk, no split combine
+    """Kernels of this library one step launches: indexer, top-k and attention
+    (the split-K combine runs inside the attention kernel)."""
+    if prefill:   # three kernels per 512-row chunk
         return 3 * ((T + 511) // 512)
-    return 3 + (1 if ran & N.DSA_KERNEL_MLA_COMBINE else 0)
+    return 3
 
 
 def run_ours(args):

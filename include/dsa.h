@@ -180,7 +180,7 @@ dsa_status dsa_read_device_status(void* ws, dsa_stream_t stream, int32_t* status
 #define DSA_KERNEL_TOPK         0x04u
 #define DSA_KERNEL_MLA_SIMT     0x08u
 #define DSA_KERNEL_MLA_TC       0x10u   /* tcgen05 bf16 sparse MLA */
-#define DSA_KERNEL_MLA_COMBINE  0x20u   /* split-K combine of the sparse MLA */
+#define DSA_KERNEL_MLA_COMBINE  0x20u   /* split-K combine of the sparse MLA (inside its kernel) */
 #define DSA_KERNEL_CACHE_APPEND 0x40u   /* fused FP8 quantise + cache write */
 #define DSA_KERNEL_OUT_PROJ     0x80u   /* tcgen05 output projection GEMM */
 #define DSA_KERNEL_OUT_PROJ_REDUCE 0x100u   /* split-K sum of the W_out product */

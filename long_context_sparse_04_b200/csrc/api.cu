@@ -298,8 +298,10 @@ MlaArgs mla_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* c, const
   a.lse = lse;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
   a.splits = p.splits;
-  a.part_o = reinterpret_cast<float*>(at(ws, p.mla));
-  a.part_ml = a.part_o + (size_t)r->num_rows * p.splits * d->n_heads * d->d_c;
+  a.part_o = at(ws, p.mla);
+  a.part_ml = reinterpret_cast<float*>(
+      at(ws, p.mla + (size_t)r->num_rows * p.splits * d->n_heads * d->d_c * sizeof(float)));
+  a.part_cnt = reinterpret_cast<unsigned long long*>(a.part_ml + (size_t)r->num_rows * p.splits * d->n_heads * 4);
   a.trace = trace_buffer() ? trace_buffer() + kTraceMla : nullptr;
   return a;
 }
@@ -313,7 +315,8 @@ dsa_status run_mla(const dsa_dims* d, MlaArgs& a, cudaStream_t s) {
 // by the split-K partials, laid out as the caller workspace of
 // dsa_sparse_mla_fwd.  20 MiB holds every split plan of the tensor-core path
 // (H = 128, d_c = 512) on a 148-SM device: one CTA pair per (row, split), so
-// rows * splits <= 74, 74 * 128 * 2064 bytes = 18.6 MiB.
+// rows * splits <= 74, 74 * 128 * 2064 bytes = 18.6 MiB (plus 16 bytes of
+// arrival tickets per row).
 constexpr size_t kNoAllocScratchBytes = size_t(20) << 20;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 

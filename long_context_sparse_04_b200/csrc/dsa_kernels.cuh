@@ -55,8 +55,11 @@ struct MlaArgs {
   float* lse;                 // [T, H] or null
   DeviceStatus* status;
   // split-K scratch (tensor-core path)
-  float* part_o;              // [T, splits, H, d_c]
-  float* part_ml;             // [T, splits, H, 2]  (max, sum)
+  void* part_o;               // [T, splits, 2 ranks, 64, H] float4: unnormalised O, dims
+                              // 4i..4i+3 of the rank's 256 for head h
+  float* part_ml;             // [T, splits, 2, H, 2]  (max, sum) per CTA of the pair
+  unsigned long long* part_cnt;   // [T, 2] arrival tickets: launch id << 32 | arrivals
+  uint32_t launch_id;         // nonzero, distinct for consecutive launches
   int splits;
   long long* trace;           // profiling stamps or null
 };

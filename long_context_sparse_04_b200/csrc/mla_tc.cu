@@ -52,6 +52,7 @@ constexpr int kH = 128, kDC = 512, kDR = 64, kD = kDC + kDR;
 constexpr int kBlk = 64;
 constexpr int kNS = 3;
 constexpr int kMaxKeys = 2048;
+constexpr int kMaxSplits = 8;                 // key splits of a decode row, a power of 2
 constexpr int kGatherWarp0 = 1, kGatherWarps = 15;
 constexpr int kGatherThreads = 32 * kGatherWarps;       // 480
 constexpr int kExWarp0 = 16;                            // warps 16-19
@@ -61,6 +62,7 @@ constexpr int kRegsLaunch = 72, kRegsLow = 48, kRegsHigh = 104;
 static_assert(4 * 128 * kRegsLow + 3 * 128 * kRegsHigh <= kThreads * kRegsLaunch,
               "register split exceeds the launch's registers");
 static_assert(kThreads * kRegsLaunch <= 65536, "launch registers exceed the SM's");
+static_assert(kThreads % 32 == 0 && (kMaxSplits & (kMaxSplits - 1)) == 0, "layout");
 constexpr int kPieces = 36;                 // 16-byte pieces of one key's 288 dims per CTA
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -82,14 +84,29 @@ struct __align__(1024) MlaSmem {
   XTile xbuf;                               // the peer's partial logits of the current block
   XTile sbuf;                               // this CTA's partial logits, bulk-copied to the peer
   int32_t rows[kMaxKeys];                   // physical cache row per selected key, -1 = none
-  unsigned long long valid[kMaxKeys / kBlk];
+  uint32_t valid[2 * kMaxKeys / kBlk];      // per 32 keys: bit i set = key i has a cache row
   float red_m[2][2][kH];                    // softmax halves: block max, [block parity][half][head]
   float red_l[2][kH];                       // softmax halves: final sums
   uint64_t q_full, x_full, x_free;
   uint64_t kv_full[kNS], kv_empty[kNS];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
   uint32_t tmem_base;
+  int last_flag;                            // this CTA merges the row's splits
 };
+
+// At the end of the kernel the merge of two key splits reuses the front of
+// shared memory: [0, 128 KB) takes the other split's partial O (Q and the
+// first two gather stages), [128 KB, 192 KB) the finished bf16 rows (the third
+// stage, the RoPE stages, Q's RoPE dims and the receive buffer).
+constexpr size_t kMergeOther = 128 * 1024, kMergeStage = 64 * 1024;
+static_assert(offsetof(MlaSmem, q) == 0 && offsetof(MlaSmem, kv) == sizeof(MlaSmem::q) &&
+                  offsetof(MlaSmem, kv_rope) == offsetof(MlaSmem, kv) + sizeof(MlaSmem::kv) &&
+                  offsetof(MlaSmem, q_rope) == offsetof(MlaSmem, kv_rope) + sizeof(MlaSmem::kv_rope) &&
+                  offsetof(MlaSmem, xbuf) == offsetof(MlaSmem, q_rope) + sizeof(MlaSmem::q_rope) &&
+                  offsetof(MlaSmem, xbuf) + sizeof(MlaSmem::xbuf) >= kMergeOther + kMergeStage &&
+                  offsetof(MlaSmem, kv) + 2 * sizeof(MlaSmem::kv[0]) == kMergeOther,
+              "merge staging layout");
+__device__ __forceinline__ uint8_t* smem_base(MlaSmem& S) { return reinterpret_cast<uint8_t*>(&S); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -139,6 +156,49 @@ __device__ __forceinline__ float2 decode_partial(uint32_t w, float m) {
   const float u0 = __uint_as_float(0x4B000000u | (w & 0xFFFFu)) - 8388608.f;
   const float u1 = __uint_as_float(0x4B000000u | (w >> 16)) - 8388608.f;
   return make_float2(fmaf(-u0, kFixInv, m), fmaf(-u1, kFixInv, m));
+}
+
+// 32 value dims of the O accumulator from tensor memory (zeros when the split
+// saw no key, whose accumulator was never written).
+__device__ __forceinline__ void load_o(uint32_t taddr, bool empty, float (&o)[32]) {
+  if (empty) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = 0.f;
+    return;
+  }
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+  tmem_wait_ld();
+}
+// f[0..8) * inv as eight bf16 (round to nearest even) in one 16-byte piece.
+__device__ __forceinline__ uint4 pack8(const float* f, float inv) {
+  return make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                    pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+}
+// Row h of the CTA's finished output tile in shared memory: 256 bf16 dims as
+// 32 pieces of 16 bytes, piece c stored at c ^ (h % 32) so that a warp's 32
+// rows hit distinct banks; o * inv are dims [8 c0, 8 c0 + 32).
+__device__ __forceinline__ void stage_bf16(uint8_t* stg, int h, int c0, const float (&o)[32], float inv) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(stg + h * 512 + (((c0 + q) ^ (h & 31)) << 4)) = pack8(&o[8 * q], inv);
+}
+// Arrival ticket of one of a row's key splits: the slot holds (launch id << 32 |
+// arrivals); a slot tagged with another launch (an earlier one, or never
+// written) counts as empty, and the last arrival resets the count, so the
+// slots need no clearing between launches.
+// Returns the arrivals of this launch, this one included (0 if the CAS loop,
+// which only ever competes with the row's other splits, were to run away).
+__device__ __forceinline__ uint32_t take_ticket(unsigned long long* slot, uint32_t id, DeviceStatus* st) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(slot);
+  for (int it = 0; it < 1 << 16; ++it) {
+    const unsigned long long nv =
+        (uint32_t)(cur >> 32) == id ? cur + 1ull : ((unsigned long long)id << 32) | 1ull;
+    const unsigned long long got = atomicCAS(slot, cur, nv);
+    if (got == cur) return (uint32_t)nv;
+    cur = got;
+  }
+  set_status(st, DSA_ERR_TIMEOUT, 29);
+  return 0u;
 }
 
 __device__ __forceinline__ void tstamp(long long* tr, uint32_t rank, int ev, int j) {
@@ -278,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int i = threadIdx.x + u * kThreads;
+      int row = -1;
       if (i < nk) {
-        int row = -1;
         const int sk = sv[u];
         if (sk >= 0 && sk < klen) {
           bool ok = true;
@@ -288,13 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
         }
         S.rows[i] = row;
       }
+      // a warp holds 32 consecutive keys (kThreads is a multiple of 32): their
+      // validity bits in one ballot
+      const uint32_t bits = __ballot_sync(0xffffffffu, row >= 0);
+      if ((threadIdx.x & 31) == 0 && (i >> 5) < 2 * nblk) S.valid[i >> 5] = bits;
     }
-  }
-  __syncthreads();
-  for (int b = threadIdx.x; b < nblk; b += kThreads) {
-    unsigned long long m = 0;
-    for (int i = 0; i < kBlk; ++i) m |= (unsigned long long)(S.rows[b * kBlk + i] >= 0) << i;
-    S.valid[b] = m;
   }
   tc_fence_before();
   __syncthreads();
@@ -411,11 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       }
       if (sidx == 0) tstamp(a.trace, rank, 0, j);
       // masked (only partial blocks) logits in the log2 domain; this half's max
-      const unsigned long long mask = S.valid[j] >> (32 * half);
-      if ((uint32_t)mask != 0xFFFFFFFFu) {
+      const uint32_t mask = S.valid[2 * j + half];
+      if (mask != 0xFFFFFFFFu) {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (!((mask >> i) & 1ull)) s[i] = -INFINITY;
+          if (!((mask >> i) & 1u)) s[i] = -INFINITY;
       }
       float pm[8];
 #pragma unroll
@@ -486,47 +544,146 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       dead = !mbar_wait(&S.pv_done[(nblk - 1) & 1], ((nblk - 1) >> 1) & 1, a.status, 27);
       tc_fence_after();
     }
-    // the row's sum over both key halves
+    // the row's sum over both key halves; a timed-out wait anywhere fails the CTA
     S.red_l[half][h] = l;
-    named_bar_sync(4, 256);
+    const bool fail = named_bar_or(4, 256, dead);
     const float lt = S.red_l[0][h] + S.red_l[1][h];
-    const bool have = __all_sync(0xffffffffu, !dead) && nblk > 0;
-    const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
+    const bool empty = nblk == 0;        // no visible key in this split: O = 0, l = 0
+    const int col0 = 128 * half;         // this thread's value dims within the CTA's 256
+    if (!fail) {
+      // The finished rows go through shared memory (the gather ring, idle once the
+      // last PV is done) so that global writes are whole 512-byte row segments.
+      uint8_t* stg = &S.kv[0][0][0];
+      bool write_out = true;
+      if (a.splits == 1) {
+        const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t o[32];
-      if (have) {
-        tmem_ld32(tmem + lane_off + kColO + 128 * half + 32 * cc, o);
-        tmem_wait_ld();
+        for (int cc = 0; cc < 4; ++cc) {
+          float o[32];
+          load_o(tmem + lane_off + kColO + col0 + 32 * cc, empty, o);
+          stage_bf16(stg, h, (col0 + 32 * cc) / 8, o, inv);
+        }
+        if (half == 0 && rank == 0 && a.lse)
+          a.lse[ro] = lt > 0.f ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
       } else {
+        // Split-K: publish this split's unnormalised O and (max, sum); the last of
+        // the row's splits to arrive (per CTA rank) merges them in split order:
+        //   out = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - M),  M = max_s m_s.
+        float4* po = reinterpret_cast<float4*>(a.part_o);
+        float2* pml = reinterpret_cast<float2*>(a.part_ml);
+        const int64_t per_unit = (256 / 4) * kH;           // float4s of one (row, split, rank)
+        const int64_t mine = (((int64_t)t * a.splits + sp) * 2 + rank) * per_unit;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float o[32];
+          load_o(tmem + lane_off + kColO + col0 + 32 * cc, empty, o);
+          const int d0 = (col0 + 32 * cc) / 4;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
-      const int dim0 = 256 * (int)rank + 128 * half + 32 * cc;
-      if (a.splits > 1) {
-        float4* dst = reinterpret_cast<float4*>(
-            a.part_o + (((int64_t)t * a.splits + sp) * kH + h) * kDC + dim0);
+          for (int i = 0; i < 8; ++i)
+            po[mine + (int64_t)(d0 + i) * kH + h] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+        if (half == 0) pml[(((int64_t)t * a.splits + sp) * 2 + rank) * kH + h] = make_float2(m_used, lt);
+        // release this CTA's partial (the barrier orders every thread's stores
+        // before thread 0's fence), then take the ticket
+        named_bar_sync(4, 256);
+        if (sidx == 0) {
+          __threadfence();
+          unsigned long long* slot = &a.part_cnt[(int64_t)t * 2 + rank];
+          const bool last = take_ticket(slot, a.launch_id, a.status) == (uint32_t)a.splits;
+          // every split has arrived: reset the count, so that a replay of the same
+          // launch (a captured graph keeps its launch id) counts from zero again
+          if (last) *slot = (unsigned long long)a.launch_id << 32;
+          S.last_flag = last;
+          __threadfence();
+        }
+        named_bar_sync(4, 256);
+        write_out = S.last_flag != 0;
+        if (write_out) {
+          if (sidx == 0 && a.status != nullptr) atomicOr(&a.status->ran, DSA_KERNEL_MLA_COMBINE);
+          float ws[kMaxSplits];
+          float M = -INFINITY, L = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                               __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ro * kDC + dim0);
+          for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+            ws[s2] = s2 < a.splits ? __ldcg(&pml[(((int64_t)t * a.splits + s2) * 2 + rank) * kH + h]).x
+                                   : -INFINITY;
+            M = fmaxf(M, ws[s2]);
+          }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float* f = reinterpret_cast<const float*>(&o[8 * i]);
-          dst[i] = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
-                              pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
+          for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+            if (s2 < a.splits) {
+              const float2 v = __ldcg(&pml[(((int64_t)t * a.splits + s2) * 2 + rank) * kH + h]);
+              ws[s2] = (v.x == -INFINITY) ? 0.f : exp2f(v.x - M);
+              L += ws[s2] * v.y;
+            } else {
+              ws[s2] = 0.f;
+            }
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          // With two splits the other one's 128 KB come into shared memory (Q and
+          // the first two gather stages, idle since the last products) in one
+          // round of copies; the finished rows are staged after them.
+          const bool staged = a.splits == 2;
+          uint8_t* other = smem_base(S);
+          if (staged) {
+            stg = smem_base(S) + kMergeOther;
+            const float4* src = po + (((int64_t)t * 2 + (sp ^ 1)) * 2 + rank) * per_unit;
+#pragma unroll 4
+            for (int k = 0; k < 32; ++k) cp_async_16(other + (sidx + 256 * k) * 16, src + sidx + 256 * k);
+            cp_async_commit();
+            cp_async_wait_all();
+            named_bar_sync(4, 256);
+          }
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            const int d0 = (col0 + 32 * cc) / 4;
+            float acc[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+              if (s2 < a.splits) {
+                const float w = ws[s2];
+                if (s2 == sp) {
+                  float o[32];
+                  load_o(tmem + lane_off + kColO + col0 + 32 * cc, empty, o);
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, o[i], acc[i]);
+                } else {
+                  const int64_t u = (((int64_t)t * a.splits + s2) * 2 + rank) * per_unit;
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const float4 v = staged ? *reinterpret_cast<const float4*>(other + ((d0 + i) * kH + h) * 16)
+                                            : __ldcg(po + u + (int64_t)(d0 + i) * kH + h);
+                    acc[4 * i] = fmaf(w, v.x, acc[4 * i]);
+                    acc[4 * i + 1] = fmaf(w, v.y, acc[4 * i + 1]);
+                    acc[4 * i + 2] = fmaf(w, v.z, acc[4 * i + 2]);
+                    acc[4 * i + 3] = fmaf(w, v.w, acc[4 * i + 3]);
+                  }
+                }
+              }
+            }
+            stage_bf16(stg, h, (col0 + 32 * cc) / 8, acc, inv);
+          }
+          if (half == 0 && rank == 0 && a.lse)
+            a.lse[ro] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
         }
       }
-    }
-    if (half == 0 && (a.splits > 1 || rank == 0)) {
-      if (a.splits > 1) {
-        reinterpret_cast<float2*>(a.part_ml)[(((int64_t)t * a.splits + sp) * 2 + rank) * kH + h] =
-            make_float2(m_used, lt);
-      } else if (a.lse) {
-        a.lse[ro] = lt > 0.f ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
+      if (write_out) {
+        named_bar_sync(4, 256);
+        // 128 rows x 32 pieces of 16 bytes; a warp writes one row's 512 bytes
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + (int64_t)t * kH * kDC + 256 * rank;
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+          const int i = sidx + 256 * k, row = i >> 5, ch = i & 31;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 512 + ((ch ^ (row & 31)) << 4));
+          reinterpret_cast<uint4*>(out + (int64_t)row * kDC)[ch] = v;
+        }
       }
+    } else {
+      // a bounded wait ran out (recorded in the status word): zeros
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ro * kDC + 256 * rank + col0);
+#pragma unroll 1
+      for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   tc_fence_before();
@@ -536,37 +693,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-}
-
-// out[t,h,:] = sum_s w_s O_s / sum_s w_s l_s,  w_s = 2^(m_s - max_s m_s); fixed split order.
-__global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
-  // thread i: value dims 4i..4i+3, produced by CTA rank (4i >= 256) with that
-  // CTA's own softmax state (m, l) of each split
-  pdl_wait();                                // the partials come from the attention kernel
-  trace_kernel(a.status, DSA_KERNEL_MLA_COMBINE);
-  const int th = blockIdx.x;
-  const int t = th / kH, h = th % kH;
-  const int r = threadIdx.x >= 64 ? 1 : 0;
-  const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
-  auto at = [&](int s) { return ml[(((int64_t)t * a.splits + s) * 2 + r) * kH + h]; };
-  float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, at(s).x);
-  float L = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < a.splits; ++s) {
-    const float2 v = at(s);
-    const float w = (v.x == -INFINITY) ? 0.f : exp2f(v.x - M);
-    L += w * v.y;
-    const float4 o = reinterpret_cast<const float4*>(
-        a.part_o + (((int64_t)t * a.splits + s) * kH + h) * kDC)[threadIdx.x];
-    acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  uint2 pk;
-  pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-  pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-  reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + ((int64_t)t * kH + h) * kDC)[threadIdx.x] = pk;
-  if (threadIdx.x == 0 && a.lse) a.lse[(int64_t)t * kH + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 
 }  // namespace
@@ -581,13 +707,16 @@ int mla_tc_splits(int num_rows) {
   if (num_rows <= 0) return 1;
   const int pairs = device_sm_count() / 2;
   int s = 1;
-  while (s < 8 && (int64_t)num_rows * s * 2 <= pairs) s <<= 1;
+  while (s < kMaxSplits && (int64_t)num_rows * s * 2 <= pairs) s <<= 1;
   return s;
 }
 
+// Split-K scratch: partial O (fp32) and (max, sum) per (row, split, head), then
+// one 8-byte arrival ticket per (row, CTA rank).
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits) {
   if (splits <= 1) return 0;
-  return (size_t)num_rows * splits * n_heads * (d_c * sizeof(float) + 4 * sizeof(float));
+  return (size_t)num_rows * splits * n_heads * (d_c * sizeof(float) + 4 * sizeof(float)) +
+         (size_t)num_rows * 2 * sizeof(unsigned long long);
 }
 
 static_assert(sizeof(MlaSmem) + 1024 <= 227 * 1024, "shared memory of the attention kernel");
@@ -640,26 +769,14 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   attr2[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr2;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, a, keys_per_split);
+  // a launch id for the split arrival tickets: distinct for consecutive launches, never 0
+  static std::atomic<uint32_t> launch_seq{0};
+  MlaArgs la = a;
+  do la.launch_id = launch_seq.fetch_add(1u) + 1u; while (la.launch_id == 0u);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, la, keys_per_split);
   if (e != cudaSuccess) {
     set_error("mla_tc launch: %s", cudaGetErrorString(e));
     return DSA_ERR_CUDA;
-  }
-  if (a.splits > 1) {
-    cudaLaunchConfig_t cc = {};
-    cc.gridDim = dim3((unsigned)(a.num_rows * kH));
-    cc.blockDim = dim3(128);
-    cc.stream = stream;
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cc.attrs = pdl;
-    cc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cc, mla_combine_kernel, a);
-    if (e != cudaSuccess) {
-      set_error("mla_combine launch: %s", cudaGetErrorString(e));
-      return DSA_ERR_CUDA;
-    }
   }
   return DSA_OK;
 }

@@ -128,3 +128,43 @@ def test_block_table_out_of_range_is_reported(N):
     torch.cuda.synchronize()
     st, det = wl.status(N.DSA_OP_INDEXER)
     assert st == N.DSA_ERR_OUT_OF_RANGE and det == cache["num_pages"] + 7
+
+
+def test_split_merge_on_a_reused_workspace(N):
+    """The key splits of a decode row are merged inside the attention kernel by
+    the last split to arrive, counted through arrival tickets in the workspace.
+    A workspace holding stale bytes, reused by calls with different split plans
+    and by repeated calls, gives the bits of a freshly initialised one."""
+    import torch
+    from long_context_sparse_04_b200.workload import DeviceWorkload, _vp
+
+    wl = DeviceWorkload(I.generate(SMALL["paged_small"]))
+    idx = wl.topk_(wl.indexer())
+    torch.cuda.synchronize()
+    need = {k: N.dsa_workspace_size(wl.dims, N.dsa_rows(
+        num_rows=k, row_seq=_vp(wl.row_seq), row_klen=_vp(wl.row_klen),
+        max_klen=wl.max_klen, q_group=wl.rows.q_group), N.DSA_OP_SPARSE_MLA) for k in (1, 3, 8)}
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    stale = torch.randint(0, 256, (max(need.values()),), dtype=torch.uint8, device="cuda",
+                          generator=gen)
+    N.dsa_workspace_init(_vp(stale), 256, wl.stream)          # the status block only
+    for k in (8, 1, 3, 8, 3):
+        rows = N.dsa_rows(num_rows=k, row_seq=_vp(wl.row_seq), row_klen=_vp(wl.row_klen),
+                          max_klen=wl.max_klen, q_group=wl.rows.q_group)
+        fresh = torch.empty(need[k], dtype=torch.uint8, device="cuda")
+        N.dsa_workspace_init(_vp(fresh), need[k], wl.stream)
+        outs = []
+        for ws in (fresh, stale):
+            out = torch.full((k, wl.H, wl.d_c), float("nan"), dtype=torch.bfloat16, device="cuda")
+            lse = torch.full((k, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+            N.dsa_sparse_mla_fwd(wl.dims, rows, wl.cache, _vp(wl.q), _vp(idx), _vp(out), _vp(lse),
+                                 _vp(ws), need[k], wl.stream)
+            assert N.dsa_read_device_status(_vp(ws), wl.stream) == (0, -1)
+            ran = N.dsa_read_kernel_trace(_vp(ws), wl.stream)
+            assert ran & N.DSA_KERNEL_MLA_TC, hex(ran)
+            # a plan with key splits merges them (and says so)
+            assert bool(ran & N.DSA_KERNEL_MLA_COMBINE) == (need[k] > 256), (k, hex(ran))
+            outs.append((out, lse))
+        assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16)), k
+        assert torch.equal(outs[0][1].view(torch.int32), outs[1][1].view(torch.int32)), k
+        assert not torch.isnan(outs[1][0].float()).any(), k
