@@ -61,6 +61,7 @@ struct MlaArgs {
   unsigned long long* part_cnt;   // [T, 2] arrival tickets: launch id << 32 | arrivals
   uint32_t launch_id;         // nonzero, distinct for consecutive launches
   int splits;
+  int merge_in_cluster;       // 2 splits in one 4-CTA cluster, merged through shared memory
   long long* trace;           // profiling stamps or null
 };
 

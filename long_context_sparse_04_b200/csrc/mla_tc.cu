@@ -88,25 +88,24 @@ struct __align__(1024) MlaSmem {
   float red_m[2][2][kH];                    // softmax halves: block max, [block parity][half][head]
   float red_l[2][kH];                       // softmax halves: final sums
   uint64_t q_full, x_full, x_free;
+  uint64_t m_ready, m_full;                 // split merge in a 4-CTA cluster
   uint64_t kv_full[kNS], kv_empty[kNS];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
   uint32_t tmem_base;
   int last_flag;                            // this CTA merges the row's splits
 };
 
-// At the end of the kernel the merge of two key splits reuses the front of
-// shared memory: [0, 128 KB) takes the other split's partial O (Q and the
-// first two gather stages), [128 KB, 192 KB) the finished bf16 rows (the third
-// stage, the RoPE stages, Q's RoPE dims and the receive buffer).
-constexpr size_t kMergeOther = 128 * 1024, kMergeStage = 64 * 1024;
-static_assert(offsetof(MlaSmem, q) == 0 && offsetof(MlaSmem, kv) == sizeof(MlaSmem::q) &&
-                  offsetof(MlaSmem, kv_rope) == offsetof(MlaSmem, kv) + sizeof(MlaSmem::kv) &&
-                  offsetof(MlaSmem, q_rope) == offsetof(MlaSmem, kv_rope) + sizeof(MlaSmem::kv_rope) &&
-                  offsetof(MlaSmem, xbuf) == offsetof(MlaSmem, q_rope) + sizeof(MlaSmem::q_rope) &&
-                  offsetof(MlaSmem, xbuf) + sizeof(MlaSmem::xbuf) >= kMergeOther + kMergeStage &&
-                  offsetof(MlaSmem, kv) + 2 * sizeof(MlaSmem::kv[0]) == kMergeOther,
-              "merge staging layout");
 __device__ __forceinline__ uint8_t* smem_base(MlaSmem& S) { return reinterpret_cast<uint8_t*>(&S); }
+// The split merge inside a 4-CTA cluster: each CTA of a pair keeps 128 of its
+// 256 value dims and receives the other split's partial O of them (64 KB fp32,
+// into Q's space) and its (max, sum) per head; it sends the other 128 from
+// the first two gather stages.  The finished bf16 rows are staged in the third.
+constexpr size_t kRecvO = 0, kSendO = 64 * 1024, kStage4 = 128 * 1024;
+constexpr size_t kSendMl = 160 * 1024, kRecvMl = 161 * 1024;
+constexpr uint32_t kMergeO = 64 * 1024, kMergeMl = kH * 8, kMergeTx = kMergeO + kMergeMl;
+static_assert(offsetof(MlaSmem, kv) == kSendO && offsetof(MlaSmem, kv) + 2 * sizeof(MlaSmem::kv[0]) == kStage4 &&
+                  offsetof(MlaSmem, kv_rope) == kSendMl && kRecvMl + kMergeMl <= kSendMl + sizeof(MlaSmem::kv_rope),
+              "cluster merge layout");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -268,7 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   MlaSmem& S = *reinterpret_cast<MlaSmem*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                            ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
-  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  // CTA rank r of the pair holds dims half r; with the split merge in the
+  // cluster, ranks 2 and 3 are the second split's pair
+  const uint32_t crank = cluster_ctarank(), rank = crank & 1u, peer = crank ^ 1u;
   const int unit = blockIdx.x >> 1;
   const int t = unit / a.splits, sp = unit % a.splits;
   pdl_launch_dependents();
@@ -282,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     mbar_init(&S.q_full, kGatherThreads);
     mbar_init(&S.x_full, 1);                 // armed by this CTA, completed by the peer's copy
     mbar_init(&S.x_free, 1);                 // the peer's receive buffer is free
+    mbar_init(&S.m_ready, 1);                // the other split's CTA can take its half
+    mbar_init(&S.m_full, 1);                 // this CTA's half of the other split landed
     for (int i = 0; i < kNS; ++i) {
       mbar_init(&S.kv_full[i], kGatherThreads);
       mbar_init(&S.kv_empty[i], 1);
@@ -308,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   const int nblk = (nvalid + kBlk - 1) / kBlk;
   const int seq = a.row_seq[t];
   if (threadIdx.x == 0 && nblk > 0) mbar_expect_tx(&S.x_full, kXBytes);   // arm the first transfer
+  if (threadIdx.x == 0 && a.merge_in_cluster) mbar_expect_tx(&S.m_full, kMergeTx);
   const bool gather_warp = warp >= kGatherWarp0 && warp < kGatherWarp0 + kGatherWarps;
   const int g = threadIdx.x - 32 * kGatherWarp0;          // gather thread index (0..479)
   // Q first: its pieces land while the selection is resolved below (the
@@ -550,7 +554,92 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     const float lt = S.red_l[0][h] + S.red_l[1][h];
     const bool empty = nblk == 0;        // no visible key in this split: O = 0, l = 0
     const int col0 = 128 * half;         // this thread's value dims within the CTA's 256
-    if (!fail) {
+    if (a.merge_in_cluster) {
+      // Two key splits in one 4-CTA cluster: the CTA of split s keeps value dims
+      // [128 s, 128 s + 128) of its rank's 256, receives the other split's
+      // partial O of them and (max, sum) through shared memory, and sends that
+      // split's CTA of the same rank (cluster rank crank ^ 2) the other 128.
+      // Every CTA takes part in the exchange, also after a timed-out wait, so
+      // that its partner's waits end.
+      const uint32_t partner = crank ^ 2u;
+      uint8_t* base = smem_base(S);
+      const int keep0 = 128 * sp, send0 = 128 * (sp ^ 1);
+      // this CTA's receive area (Q's space) is free: its last products are done
+      if (sidx == 0) mbar_arrive_cluster(&S.m_ready, partner);
+      float4* send = reinterpret_cast<float4*>(base + kSendO);
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        float o[32];
+        load_o(tmem + lane_off + kColO + send0 + 64 * half + 32 * cc, empty || fail, o);
+        const int d0 = (64 * half + 32 * cc) / 4;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          send[(d0 + i) * kH + h] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      }
+      if (half == 0) reinterpret_cast<float2*>(base + kSendMl)[h] = make_float2(m_used, lt);
+      fence_proxy_async_smem();            // generic writes -> bulk copy engine
+      named_bar_sync(4, 256);
+      if (sidx == 0 && mbar_wait_cluster(&S.m_ready, 0, a.status, 30)) {
+        bulk_copy_to_peer(base + kRecvO, base + kSendO, kMergeO, &S.m_full, partner);
+        bulk_copy_to_peer(base + kRecvMl, base + kSendMl, kMergeMl, &S.m_full, partner);
+        bulk_commit();
+        bulk_wait_read0();
+      }
+      const bool got = mbar_wait_cluster(&S.m_full, 0, a.status, 31);
+      const bool bad = named_bar_or(4, 256, fail || !got);
+      if (!bad) {
+        // out = (w0 O_0 + w1 O_1) / (w0 l_0 + w1 l_1), w_s = 2^(m_s - M), split 0 first
+        const float2 mine = make_float2(m_used, lt);
+        const float2 theirs = reinterpret_cast<const float2*>(base + kRecvMl)[h];
+        const float2 s0 = sp == 0 ? mine : theirs, s1 = sp == 0 ? theirs : mine;
+        const float M = fmaxf(s0.x, s1.x);
+        const float w0 = s0.x == -INFINITY ? 0.f : exp2f(s0.x - M);
+        const float w1 = s1.x == -INFINITY ? 0.f : exp2f(s1.x - M);
+        const float L = fmaf(w1, s1.y, w0 * s0.y);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float4* recv = reinterpret_cast<const float4*>(base + kRecvO);
+        uint8_t* stg4 = base + kStage4;     // 128 rows x 256 bytes, pieces swizzled by row
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          float own[32], acc[32];
+          load_o(tmem + lane_off + kColO + keep0 + 64 * half + 32 * cc, empty, own);
+          const int d0 = (64 * half + 32 * cc) / 4;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = recv[(d0 + i) * kH + h];
+            const float r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = sp == 0 ? own[4 * i + e] : r[e];
+              const float x1 = sp == 0 ? r[e] : own[4 * i + e];
+              acc[4 * i + e] = fmaf(w1, x1, w0 * x0);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int c = (64 * half + 32 * cc) / 8 + q;
+            *reinterpret_cast<uint4*>(stg4 + h * 256 + ((c ^ (h & 15)) << 4)) = pack8(&acc[8 * q], inv);
+          }
+        }
+        if (half == 0 && rank == 0 && sp == 0 && a.lse)
+          a.lse[ro] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        named_bar_sync(4, 256);
+        // 128 rows x 16 pieces of 16 bytes; a half warp writes one row's 256 bytes
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + (int64_t)t * kH * kDC + 256 * rank + keep0;
+#pragma unroll 4
+        for (int k = 0; k < 8; ++k) {
+          const int i = sidx + 256 * k, row = i >> 4, ch = i & 15;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg4 + row * 256 + ((ch ^ (row & 15)) << 4));
+          reinterpret_cast<uint4*>(out + (int64_t)row * kDC)[ch] = v;
+        }
+      } else {
+        // a bounded wait ran out (recorded in the status word): zeros
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + ro * kDC + 256 * rank +
+                                              keep0 + 64 * half);
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else if (!fail) {
       // The finished rows go through shared memory (the gather ring, idle once the
       // last PV is done) so that global writes are whole 512-byte row segments.
       uint8_t* stg = &S.kv[0][0][0];
@@ -619,20 +708,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
             }
           }
           const float inv = L > 0.f ? 1.f / L : 0.f;
-          // With two splits the other one's 128 KB come into shared memory (Q and
-          // the first two gather stages, idle since the last products) in one
-          // round of copies; the finished rows are staged after them.
-          const bool staged = a.splits == 2;
-          uint8_t* other = smem_base(S);
-          if (staged) {
-            stg = smem_base(S) + kMergeOther;
-            const float4* src = po + (((int64_t)t * 2 + (sp ^ 1)) * 2 + rank) * per_unit;
-#pragma unroll 4
-            for (int k = 0; k < 32; ++k) cp_async_16(other + (sidx + 256 * k) * 16, src + sidx + 256 * k);
-            cp_async_commit();
-            cp_async_wait_all();
-            named_bar_sync(4, 256);
-          }
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             const int d0 = (col0 + 32 * cc) / 4;
@@ -652,8 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
                   const int64_t u = (((int64_t)t * a.splits + s2) * 2 + rank) * per_unit;
 #pragma unroll
                   for (int i = 0; i < 8; ++i) {
-                    const float4 v = staged ? *reinterpret_cast<const float4*>(other + ((d0 + i) * kH + h) * 16)
-                                            : __ldcg(po + u + (int64_t)(d0 + i) * kH + h);
+                    const float4 v = __ldcg(po + u + (int64_t)(d0 + i) * kH + h);
                     acc[4 * i] = fmaf(w, v.x, acc[4 * i]);
                     acc[4 * i + 1] = fmaf(w, v.y, acc[4 * i + 1]);
                     acc[4 * i + 2] = fmaf(w, v.z, acc[4 * i + 2]);
@@ -747,6 +821,35 @@ dsa_status check_register_split() {
   return DSA_OK;
 }
 
+// Clusters of four attention CTAs that can be resident at once on this device
+// (0 if the query fails), looked up once per device.
+int max_merge_clusters(size_t smem) {
+  static std::atomic<int> cached[kMaxDevices];
+  static std::atomic<bool> have[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (have[dev].load()) return cached[dev].load();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(4);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 4;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cached[dev].store(n);
+  have[dev].store(true);
+  return n;
+}
+
 dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
   const size_t smem = sizeof(MlaSmem) + 1024;
@@ -760,9 +863,13 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
+  // Two key splits of a row run as one 4-CTA cluster and merge through shared
+  // memory when every cluster of the grid can be resident at once.
+  MlaArgs la = a;
+  la.merge_in_cluster = a.splits == 2 && a.num_rows <= max_merge_clusters(smem) ? 1 : 0;
   cudaLaunchAttribute attr2[2];
   attr2[0].id = cudaLaunchAttributeClusterDimension;
-  attr2[0].val.clusterDim.x = 2;
+  attr2[0].val.clusterDim.x = la.merge_in_cluster ? 4 : 2;
   attr2[0].val.clusterDim.y = 1;
   attr2[0].val.clusterDim.z = 1;
   attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -771,7 +878,6 @@ dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream) {
   cfg.numAttrs = 2;
   // a launch id for the split arrival tickets: distinct for consecutive launches, never 0
   static std::atomic<uint32_t> launch_seq{0};
-  MlaArgs la = a;
   do la.launch_id = launch_seq.fetch_add(1u) + 1u; while (la.launch_id == 0u);
   cudaError_t e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, la, keys_per_split);
   if (e != cudaSuccess) {
