@@ -629,6 +629,36 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
 
 size_t topk_ws_bytes() { return 0; }
 
+// Clusters of `csize` CTAs of `fn` that can be resident at once (0 if the
+// query fails), looked up once per device, instantiation and cluster size.
+int max_topk_clusters(const void* fn, int which, int csize, size_t smem) {
+  static std::atomic<int> cached[2][4][kMaxDevices];
+  static std::atomic<bool> have[2][4][kMaxDevices];
+  const int ci = csize >= 8 ? 3 : csize >= 4 ? 2 : csize >= 2 ? 1 : 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (have[which][ci][dev].load()) return cached[which][ci][dev].load();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)csize);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = csize;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cached[which][ci][dev].store(n);
+  have[which][ci][dev].store(true);
+  return n;
+}
+
 dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
   int csize = 1;
@@ -651,7 +681,13 @@ dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  // A programmatic launch places the clusters while the previous kernel's last
+  // CTAs still hold SMs; clusters of four or more CTAs placed piecemeal pack
+  // worse, and a grid that fits the device in one wave of clusters may then
+  // need two.  Such a grid is launched once the previous kernel is done.
+  const bool one_wave =
+      csize >= 4 && a.num_rows <= max_topk_clusters(fn, a.hist ? 1 : 0, csize, smem);
+  cfg.numAttrs = one_wave ? 1 : 2;
   cudaError_t e = a.hist ? cudaLaunchKernelEx(&cfg, topk_kernel<true>, a)
                          : cudaLaunchKernelEx(&cfg, topk_kernel<false>, a);
   if (e != cudaSuccess) {
