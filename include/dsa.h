@@ -164,7 +164,10 @@ size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op)
  * score histograms of the fused indexer -> top-k, which every top-k leaves
  * zeroed for the next call.  Call it once before the first use of a
  * workspace, and again after a call that recorded a device error (a call cut
- * short may leave histograms behind). */
+ * short may leave histograms behind).  A workspace may then serve calls of
+ * other ops or other rows in any order: the library records, per workspace
+ * address on the host, which bytes its calls left zeroed, and a call whose
+ * histogram region is not among them clears it first (one memset). */
 dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /* Synchronise `stream`, copy the device status word of `ws` to *status_out

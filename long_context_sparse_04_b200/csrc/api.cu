@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "dsa_kernels.cuh"
 
@@ -273,6 +274,38 @@ dsa_status run_indexer(const dsa_dims* d, IndexerArgs& a, void* ws, const WsPlan
 
 // The fused indexer -> top-k: the indexer builds each row's histogram of its
 // scores' top 12 key bits, and top-k starts from it.
+// Which bytes of a workspace are known to be zero, per workspace address: all
+// of it after dsa_workspace_init, the histogram region after a call whose
+// top-k cleared it, nothing after any other call that writes the workspace.
+// The fused histograms are accumulated into, so a call whose histogram region
+// is not vouched for (a workspace reused with other rows or another op, whose
+// data may lie there) clears it first.
+struct ZeroSpan {
+  size_t off = 0, bytes = 0;
+};
+std::mutex g_zero_mu;
+std::unordered_map<const void*, ZeroSpan> g_zero;
+
+void ws_zero_set(const void* ws, size_t off, size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_zero_mu);
+  g_zero[ws] = ZeroSpan{off, bytes};
+}
+void ws_zero_forget(const void* ws) { ws_zero_set(ws, 0, 0); }
+bool ws_zero_covers(const void* ws, size_t off, size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_zero_mu);
+  const auto it = g_zero.find(ws);
+  return it != g_zero.end() && it->second.off <= off && off + bytes <= it->second.off + it->second.bytes;
+}
+// Before a fused call: the histogram region is zero (cleared now if not vouched for).
+dsa_status ws_hist_ready(void* ws, const WsPlan& p, cudaStream_t s) {
+  if (ws_zero_covers(ws, p.hist, p.hist_bytes)) return DSA_OK;
+  if (cudaMemsetAsync(at(ws, p.hist), 0, p.hist_bytes, s) != cudaSuccess) {
+    set_error("clearing the histogram region failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
 uint32_t* fused_hist(const dsa_dims* d, const IndexerArgs& ia, void* ws, const WsPlan& p) {
   if (d->algo != DSA_ALGO_AUTO || p.hist_bytes == 0 || !indexer_tc_hist_supported(ia)) return nullptr;
   return reinterpret_cast<uint32_t*>(at(ws, p.hist));
@@ -383,6 +416,7 @@ dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream) {
     set_error("cudaMemsetAsync failed");
     return DSA_ERR_CUDA;
   }
+  ws_zero_set(ws, 0, ws_bytes);
   return DSA_OK;
 }
 
@@ -475,6 +509,7 @@ dsa_status dsa_indexer_scores(const dsa_dims* dims, const dsa_rows* rows, const 
   const WsPlan p = plan(dims, rows, DSA_OP_INDEXER);
   if ((st = check_ws(ws, ws_bytes, p.total))) return st;
   IndexerArgs a = indexer_args(dims, rows, cache, q_idx, q_scale, w, scores, ld_scores, ws, p);
+  ws_zero_forget(ws);
   return run_indexer(dims, a, ws, p, (cudaStream_t)stream);
 }
 
@@ -500,6 +535,7 @@ dsa_status dsa_topk(const dsa_dims* dims, const dsa_rows* rows, const float* sco
   a.idx = idx;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
   a.trace = trace_buffer() ? trace_buffer() + kTraceTopk : nullptr;
+  ws_zero_forget(ws);
   return launch_topk(a, rows->max_klen, (cudaStream_t)stream);
 }
 
@@ -517,6 +553,7 @@ dsa_status dsa_sparse_mla_fwd(const dsa_dims* dims, const dsa_rows* rows, const 
   const WsPlan p = plan(dims, rows, DSA_OP_SPARSE_MLA);
   if ((st = check_ws(ws, ws_bytes, p.total))) return st;
   MlaArgs a = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
+  ws_zero_forget(ws);
   return run_mla(dims, a, (cudaStream_t)stream);
 }
 
@@ -544,6 +581,7 @@ dsa_status dsa_sparse_mla_fwd_noalloc(const dsa_dims* dims, const dsa_rows* rows
     return DSA_ERR_CUDA;
   }
   MlaArgs a = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
+  ws_zero_forget(ws);
   return run_mla(dims, a, (cudaStream_t)stream);
 }
 
@@ -569,6 +607,8 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   int32_t* idx = dbg_idx ? dbg_idx : reinterpret_cast<int32_t*>(at(ws, p.idx));
   IndexerArgs ia = indexer_args(dims, rows, cache, q_idx, q_scale, w, scores, p.ld, ws, p);
   ia.hist = fused_hist(dims, ia, ws, p);
+  if (ia.hist && (st = ws_hist_ready(ws, p, s))) return st;
+  ws_zero_forget(ws);
   stage_event(0, s);
   if ((st = run_indexer(dims, ia, ws, p, s))) return st;
   stage_event(1, s);
@@ -587,6 +627,8 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   MlaArgs ma = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
   st = run_mla(dims, ma, s);
   stage_event(3, s);
+  // the top-k left the histogram region zeroed
+  if (st == DSA_OK && ia.hist) ws_zero_set(ws, p.hist, p.hist_bytes);
   return st;
 }
 
@@ -614,6 +656,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
   const size_t mla_el = dims->mla_dtype == DSA_BF16 ? 2 : 4;
   float* scores = reinterpret_cast<float*>(at(ws, p.scores));
   int32_t* idx_ws = reinterpret_cast<int32_t*>(at(ws, p.idx));
+  bool used_hist = false;
   for (int r0 = 0; r0 < T; r0 += p.chunk_rows) {
     const int n = (T - r0) < p.chunk_rows ? (T - r0) : p.chunk_rows;
     dsa_rows cr = *rows;
@@ -629,6 +672,9 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     int32_t* idx = idx_out ? idx_out + (size_t)r0 * dims->topk : idx_ws;
     IndexerArgs ia = indexer_args(dims, &cr, cache, qi, qs, wr, scores, p.ld, ws, p);
     ia.hist = fused_hist(dims, ia, ws, p);
+    if (ia.hist && !used_hist && (st = ws_hist_ready(ws, p, s))) return st;
+    if (r0 == 0) ws_zero_forget(ws);
+    used_hist = used_hist || ia.hist != nullptr;
     if ((st = run_indexer(dims, ia, ws, p, s))) return st;
     TopkArgs ta{};
     ta.num_rows = n;
@@ -644,6 +690,8 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     MlaArgs ma = mla_args(dims, &cr, cache, qq, idx, oo, ll, ws, p);
     if ((st = run_mla(dims, ma, s))) return st;
   }
+  // every chunk's top-k left the histogram region zeroed
+  if (used_hist) ws_zero_set(ws, p.hist, p.hist_bytes);
   return DSA_OK;
 }
 
@@ -742,6 +790,7 @@ dsa_status dsa_indexer_backward(const dsa_dims* dims, const dsa_rows* rows, cons
   a.dw = dw;
   a.dk = dk;
   a.partial = reinterpret_cast<float*>(at(ws, p.bwd));
+  ws_zero_forget(ws);
   a.chunk_keys = kWarmupChunkKeys;
   a.n_chunks = (rows->max_klen + kWarmupChunkKeys - 1) / kWarmupChunkKeys;
   a.status = reinterpret_cast<DeviceStatus*>(ws);
@@ -765,6 +814,7 @@ dsa_status dsa_output_projection(const dsa_proj_dims* dims, int32_t num_rows, co
   CHECK_ARG(num_rows >= 0, "num_rows must be >= 0");
   if ((st = check_ws(ws, ws_bytes, kStatusBytes + proj_partial_bytes(dims, num_rows))) != DSA_OK)
     return st;
+  ws_zero_forget(ws);
   if (num_rows == 0) return DSA_OK;
   CHECK_ARG(o && w_uv && w_out && u && y, "a tensor pointer is NULL");
   CHECK_ARG(aligned(o, 16) && aligned(w_uv, 16) && aligned(w_out, 16) && aligned(u, 16) &&

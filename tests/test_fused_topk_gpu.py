@@ -114,3 +114,50 @@ def test_fused_ties_and_signed_zeros(N):
 def _oracle_scores(inp, t):
     from oracle import dsa_ref as R
     return R.row_scores(inp, t)
+
+
+def test_workspace_reused_across_plans(N):
+    """One workspace serves decode steps of different row counts with other
+    ops in between, whose data lands where a later step keeps its histograms;
+    every step gives the bits of a step on a freshly initialised workspace
+    (the library clears a histogram region it cannot vouch for)."""
+    import torch
+    from long_context_sparse_04_b200.workload import DeviceWorkload, _vp
+
+    wl = DeviceWorkload(_inputs("paged_small"))
+    assert wl.rows.q_group == 2
+    big = max(N.dsa_workspace_size(wl.dims, wl.rows, op)
+              for op in (N.DSA_OP_DECODE_STEP, N.DSA_OP_INDEXER, N.DSA_OP_SPARSE_MLA))
+    shared = torch.empty(big, dtype=torch.uint8, device="cuda")
+    N.dsa_workspace_init(_vp(shared), big, wl.stream)
+
+    def rows_of(k):
+        return N.dsa_rows(num_rows=k, row_seq=_vp(wl.row_seq), row_klen=_vp(wl.row_klen),
+                          max_klen=wl.max_klen, q_group=2)
+
+    def step(rows, k, ws, n):
+        out = torch.full((k, wl.H, wl.d_c), float("nan"), dtype=torch.bfloat16, device="cuda")
+        lse = torch.full((k, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+        idx = torch.full((k, wl.topk), -7, dtype=torch.int32, device="cuda")
+        N.dsa_decode_step(wl.dims, rows, wl.cache, _vp(wl.q_idx), _vp(wl.q_scale), _vp(wl.w),
+                          _vp(wl.q), _vp(out), _vp(lse), None, _vp(idx), _vp(ws), n, wl.stream)
+        assert N.dsa_read_device_status(_vp(ws), wl.stream) == (0, -1)
+        return out, lse, idx
+
+    for k in (8, 4, 8, 2, 6):
+        rows = rows_of(k)
+        need = N.dsa_workspace_size(wl.dims, rows, N.DSA_OP_DECODE_STEP)
+        fresh = torch.empty(need, dtype=torch.uint8, device="cuda")
+        N.dsa_workspace_init(_vp(fresh), need, wl.stream)
+        ref = step(rows, k, fresh, need)
+        got = step(rows, k, shared, big)
+        assert torch.equal(ref[2], got[2]), k
+        assert torch.equal(ref[0].view(torch.int16), got[0].view(torch.int16)), k
+        assert torch.equal(ref[1].view(torch.int32), got[1].view(torch.int32)), k
+        # another op writes its own data over the shared workspace before the next step
+        scores = torch.empty((wl.T, wl.ld), dtype=torch.float32, device="cuda")
+        n_idx = N.dsa_workspace_size(wl.dims, wl.rows, N.DSA_OP_INDEXER)
+        N.dsa_indexer_scores(wl.dims, wl.rows, wl.cache, _vp(wl.q_idx), _vp(wl.q_scale), _vp(wl.w),
+                             _vp(scores), wl.ld, _vp(shared), n_idx, wl.stream)
+        shared[256:].random_(0, 256)      # stale bytes everywhere past the status block
+    torch.cuda.synchronize()
