@@ -29,6 +29,9 @@
 //    keys) skips the bitmap and scans the segment instead, warp w owning a
 //    contiguous range and warp ballots giving the order inside it.
 // Rows with klen <= k return 0..klen-1 then -1.
+//
+// Batches of at least two rows per SM (prefill chunks) run topk_row_kernel
+// instead (further below): one CTA per row streaming the scores, no cluster.
 #include "dsa_kernels.cuh"
 
 namespace dsa {
@@ -625,6 +628,304 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
   kstamp(a.trace, csize, rank, 8);
 }
 
+
+// ---------------------------------------------------------------------------
+// One CTA of 1024 threads per row, no cluster and no copy of the row in shared
+// memory: the scores are streamed from global memory (L2) in position order,
+// warp w owning a contiguous range of the row.
+//   1. The first-digit histogram (bits 31..20): the indexer's (kHist), read and
+//      zeroed for the next call, or one pass that builds it.  Its bin search
+//      gives B0 (the bin of the k-th largest key), the rank need0 of that key in
+//      B0 and the bin's count c0.
+//   2. One pass: per warp, the keys above bin B0 are counted and the keys of
+//      bin B0 are collected (with the warp that saw them) in shared memory.
+//   3. Two 10-bit digits over the c0 collected keys give T (the k-th largest
+//      key) and `need` (how many keys equal to T are taken, lowest positions
+//      first); the collected keys give each warp's counts of keys > T and == T.
+//      When c0 exceeds the collection's capacity (massive ties), two more
+//      passes over the row build the digit histograms and one counts per warp.
+//   4. A block-wide prefix of the warps' counts gives each warp its place in
+//      the output; a last pass writes the selected positions in order.
+// The positions come out ascending with ties going to the lower position.
+constexpr int kRowThreads = 1024;
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowGatherCap = 4096;   // keys of bin B0 collected in shared memory
+
+struct RowSmem {
+  uint32_t hist[kBins0];
+  uint32_t gather[kRowGatherCap];       // keys of bin B0
+  uint8_t gwarp[kRowGatherCap];         // the warp that collected each
+  uint32_t lhist[2][kBins];             // the last two digits
+  uint32_t wcnt[kRowWarps][4];          // per warp: above B0, in B0 and > T, == T
+  uint32_t warp_tmp[kRowWarps];
+  uint32_t sel_bin, sel_need, sel_cnt, gcount;
+};
+
+// Among 4096 first-digit bins, the bin of the need-th largest key (every
+// thread of the block gets it in S.sel_*).
+__device__ void row_search0(RowSmem& S, uint32_t need) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint4 m = reinterpret_cast<const uint4*>(S.hist)[tid];     // bins 4 tid .. 4 tid + 3
+  const uint32_t local = m.x + m.y + m.z + m.w;
+  uint32_t x = local;                                              // inclusive prefix in the warp
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) S.warp_tmp[warp] = x;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kRowWarps; ++w) {
+    const uint32_t v = S.warp_tmp[w];
+    before += (w < warp) ? v : 0u;
+    all += v;
+  }
+  uint32_t cum = all - (before + x);                               // keys in higher threads' bins
+  const uint32_t c[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+  for (int i = 3; i >= 0; --i) {
+    if (cum < need && cum + c[i] >= need) {
+      S.sel_bin = (uint32_t)(4 * tid + i);
+      S.sel_need = need - cum;
+      S.sel_cnt = c[i];
+    }
+    cum += c[i];
+  }
+  __syncthreads();
+}
+
+template <bool kHist>
+__global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smraw[];
+  RowSmem& S = *reinterpret_cast<RowSmem*>(smraw);
+  pdl_launch_dependents();
+  pdl_wait();                                // the scores come from the previous kernel
+  trace_kernel(a.status, DSA_KERNEL_TOPK);
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k = a.topk;
+  const int klen = a.row_klen[t];
+  int32_t* out = a.idx + (int64_t)t * k;
+  uint32_t* const ghist = kHist ? a.hist + (int64_t)t * kBins0 : nullptr;
+  if (klen <= k) {
+    for (int i = tid; i < k; i += kRowThreads) out[i] = i < klen ? i : -1;
+    if (kHist)
+      for (int i = tid; i < kBins0 / 4; i += kRowThreads)
+        reinterpret_cast<uint4*>(ghist)[i] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const float* row = a.scores + (int64_t)t * a.ld_scores;
+  // warp w: positions [w0, w1), w0 a multiple of 128; a round is 32 lanes x 4
+  const int per_warp = ((klen + 128 * kRowWarps - 1) / (128 * kRowWarps)) * 128;
+  const int w0 = min(warp * per_warp, klen), w1 = min(w0 + per_warp, klen);
+  const uint32_t lt = (1u << lane) - 1;
+  // four keys at position p (a multiple of 4, p < klen <= ld_scores, so the
+  // 16 bytes are inside the row); positions at or past w1 give no key
+  auto load4 = [&](int p) -> float4 { return __ldcg(reinterpret_cast<const float4*>(row + p)); };
+
+  // ---- 1. first digit
+  if (tid < kRowWarps) {
+    S.wcnt[tid][0] = S.wcnt[tid][1] = S.wcnt[tid][2] = S.wcnt[tid][3] = 0u;
+  }
+  if (tid == 0) S.gcount = 0u;
+  if (kHist) {
+    const uint4 h = __ldcg(reinterpret_cast<const uint4*>(ghist) + tid);
+    reinterpret_cast<uint4*>(S.hist)[tid] = h;
+    reinterpret_cast<uint4*>(ghist)[tid] = make_uint4(0u, 0u, 0u, 0u);   // for the next call
+  } else {
+    reinterpret_cast<uint4*>(S.hist)[tid] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int p0 = w0; p0 < w1; p0 += 4 * 128) {
+      float4 f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int p = p0 + 128 * u + 4 * lane;
+        f[u] = p < w1 ? load4(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int p = p0 + 128 * u + 4 * lane;
+        const float v[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (p + j < w1) atomicAdd(&S.hist[float_key(v[j]) >> 20], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  row_search0(S, (uint32_t)k);
+  const uint32_t B0 = S.sel_bin, need0 = S.sel_need, c0 = S.sel_cnt;
+  const bool gathered = c0 <= (uint32_t)kRowGatherCap;   // uniform over the block
+
+  // ---- 2. keys above B0 per warp; the keys of B0 collected
+  {
+    uint32_t above = 0;
+    for (int p0 = w0; p0 < w1; p0 += 4 * 128) {
+      float4 f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int p = p0 + 128 * u + 4 * lane;
+        f[u] = p < w1 ? load4(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int p = p0 + 128 * u + 4 * lane;
+        const float v[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool in = p + j < w1;
+          const uint32_t key = float_key(v[j]);
+          const uint32_t bin = key >> 20;
+          above += (in && bin > B0) ? 1u : 0u;
+          if (gathered) {
+            const bool mine = in && bin == B0;
+            const uint32_t bl = __ballot_sync(0xffffffffu, mine);
+            if (bl) {
+              uint32_t base = 0;
+              if (lane == 0) base = atomicAdd(&S.gcount, (uint32_t)__popc(bl));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              if (mine) {
+                const uint32_t slot = base + __popc(bl & lt);
+                S.gather[slot] = key;
+                S.gwarp[slot] = (uint8_t)warp;
+              }
+            }
+          }
+        }
+      }
+    }
+    above = __reduce_add_sync(0xffffffffu, above);
+    if (lane == 0) S.wcnt[warp][0] = above;
+  }
+  for (int i = tid; i < 2 * kBins; i += kRowThreads) (&S.lhist[0][0])[i] = 0u;
+  __syncthreads();
+
+  // ---- 3. T and `need`; per warp, keys of B0 above T and equal to it
+  uint32_t T, need;
+  if (gathered) {
+    for (int i = tid; i < (int)c0; i += kRowThreads) atomicAdd(&S.lhist[0][(S.gather[i] >> 10) & 1023u], 1u);
+    __syncthreads();
+    if (warp == 0) warp_search_1024(S.lhist[0], need0, &S.sel_bin, &S.sel_need);
+    __syncthreads();
+    const uint32_t p1 = (B0 << 10) | S.sel_bin, n1 = S.sel_need;
+    for (int i = tid; i < (int)c0; i += kRowThreads) {
+      const uint32_t key = S.gather[i];
+      if ((key >> 10) == p1) atomicAdd(&S.lhist[1][key & 1023u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) warp_search_1024(S.lhist[1], n1, &S.sel_bin, &S.sel_need);
+    __syncthreads();
+    T = (p1 << 10) | S.sel_bin;
+    need = S.sel_need;
+    for (int i = tid; i < (int)c0; i += kRowThreads) {
+      const uint32_t key = S.gather[i];
+      const int w = S.gwarp[i];
+      if (key > T) atomicAdd(&S.wcnt[w][1], 1u);
+      else if (key == T) atomicAdd(&S.wcnt[w][2], 1u);
+    }
+  } else {
+    // massive ties in bin B0: the last two digits and the per-warp counts by passes
+    uint32_t prefix = B0, nd = need0;
+#pragma unroll 1
+    for (int d = 0; d < 2; ++d) {
+      const int shift = 20 - 10 * d, nshift = shift - 10;
+      for (int p = w0 + 4 * lane; p < w1; p += 128) {
+        const float4 f = load4(p);
+        const float v[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t key = float_key(v[j]);
+          if (p + j < w1 && (key >> shift) == prefix) atomicAdd(&S.lhist[d][(key >> nshift) & 1023u], 1u);
+        }
+      }
+      __syncthreads();
+      if (warp == 0) warp_search_1024(S.lhist[d], nd, &S.sel_bin, &S.sel_need);
+      __syncthreads();
+      prefix = (prefix << 10) | S.sel_bin;
+      nd = S.sel_need;
+    }
+    T = prefix;
+    need = nd;
+    uint32_t gt = 0, eq = 0;
+    for (int p = w0 + 4 * lane; p < w1; p += 128) {
+      const float4 f = load4(p);
+      const float v[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t key = float_key(v[j]);
+        const bool in = p + j < w1;
+        gt += (in && (key >> 20) == B0 && key > T) ? 1u : 0u;
+        eq += (in && key == T) ? 1u : 0u;
+      }
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    if (lane == 0) {
+      S.wcnt[warp][1] = gt;
+      S.wcnt[warp][2] = eq;
+    }
+  }
+  __syncthreads();
+
+  // ---- 4. this warp's place in the output, then the ordered output pass
+  uint32_t pos = 0, eq_rank = 0;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t e = S.wcnt[w][2];
+    pos += S.wcnt[w][0] + S.wcnt[w][1] + (eq_rank >= need ? 0u : min(e, need - eq_rank));
+    eq_rank += e;
+  }
+  for (int p00 = w0; p00 < w1; p00 += 4 * 128) {
+    float4 fu[4];                            // four rounds' loads in flight
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p00 + 128 * u + 4 * lane;
+      fu[u] = p < w1 ? load4(p) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int p0 = p00 + 128 * u;
+    const int p = p0 + 4 * lane;
+    const float4 f = fu[u];
+    const float v[4] = {f.x, f.y, f.z, f.w};
+    bool gt[4], eq[4];
+    uint32_t e_before = 0, e_round = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = float_key(v[j]);
+      const bool in = p + j < w1;
+      gt[j] = in && key > T;
+      eq[j] = in && key == T;
+      const uint32_t bl = __ballot_sync(0xffffffffu, eq[j]);
+      e_before += __popc(bl & lt);
+      e_round += __popc(bl);
+    }
+    bool sel[4];
+    uint32_t r_eq = eq_rank + e_before;
+    uint32_t s_before = 0, s_round = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      sel[j] = gt[j] || (eq[j] && r_eq < need);
+      r_eq += eq[j];
+      const uint32_t bl = __ballot_sync(0xffffffffu, sel[j]);
+      s_before += __popc(bl & lt);
+      s_round += __popc(bl);
+    }
+    uint32_t q = pos + s_before;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (sel[j]) {
+        if (q < (uint32_t)k) out[q] = p + j;
+        ++q;
+      }
+    }
+    pos += s_round;
+    eq_rank += e_round;
+  }
+  }
+}
+
 }  // namespace
 
 size_t topk_ws_bytes() { return 0; }
@@ -659,8 +960,37 @@ int max_topk_clusters(const void* fn, int which, int csize, size_t smem) {
   return n;
 }
 
+// The row kernel: one CTA per row, streaming the scores.
+dsa_status launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
+  const size_t smem = sizeof(RowSmem);
+  static std::atomic<bool> attr_done[2][kMaxDevices] = {};
+  const void* fn = a.hist ? reinterpret_cast<const void*>(topk_row_kernel<true>)
+                          : reinterpret_cast<const void*>(topk_row_kernel<false>);
+  if (dsa_status st = set_smem_limit_once(fn, smem, attr_done[a.hist ? 1 : 0])) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.num_rows);
+  cfg.blockDim = dim3(kRowThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = a.hist ? cudaLaunchKernelEx(&cfg, topk_row_kernel<true>, a)
+                         : cudaLaunchKernelEx(&cfg, topk_row_kernel<false>, a);
+  if (e != cudaSuccess) {
+    set_error("topk launch: %s", cudaGetErrorString(e));
+    return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
 dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
+  // Many rows (a prefill chunk) fill the device with one CTA per row; a few
+  // long rows (decode) keep each row's scores in the shared memory of a cluster.
+  if (a.num_rows >= 2 * device_sm_count()) return launch_topk_rows(a, stream);
   int csize = 1;
   while (csize < kMaxCluster && (int64_t)csize * kCacheCap < (int64_t)max_klen) csize <<= 1;
   const size_t smem = sizeof(TopkSmem);

@@ -117,3 +117,24 @@ def test_topk_rows_beyond_the_cluster_cache(N, kind):
     got = _run(N, rows, 2048)
     for t, r in enumerate(rows):
         assert np.array_equal(got[t], R.topk_row(r.astype(np.float64), 2048)), (kind, r.shape[0])
+
+
+@pytest.mark.parametrize("k", [2048, 64])
+def test_topk_many_rows(N, k):
+    """A batch of hundreds of rows runs one CTA per row, streaming the scores
+    (the cluster kernel above runs the few-row batches): every kind of row,
+    lengths around k and well past it, and bins far over the threshold-bin
+    capacity (all_equal, crowded_bin), each against the oracle."""
+    lengths = [1, k - 1, k, k + 1, 3000, 4097, 6000, 9000, 20000]
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rows = []
+    i = 0
+    while len(rows) < 2 * sms + 8:
+        kind = KINDS[i % len(KINDS)]
+        rows += _rows(kind, [lengths[(i + j) % len(lengths)] for j in range(2)], seed=100 + i)
+        i += 1
+    got = _run(N, rows, k)
+    for t, r in enumerate(rows):
+        want = R.topk_row(r.astype(np.float64), k)
+        assert np.array_equal(got[t], want), (t, r.shape[0], np.flatnonzero(got[t] != want)[:5])
