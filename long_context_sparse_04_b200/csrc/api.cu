@@ -265,9 +265,13 @@ IndexerArgs indexer_args(const dsa_dims* d, const dsa_rows* r, const dsa_cache* 
   return a;
 }
 
+bool indexer_runs_tc(const dsa_dims* d, const IndexerArgs& a) {
+  return d->algo != DSA_ALGO_SIMT && indexer_tc_supported(a);
+}
+
 dsa_status run_indexer(const dsa_dims* d, IndexerArgs& a, void* ws, const WsPlan& p,
                        cudaStream_t s) {
-  if (d->algo != DSA_ALGO_SIMT && indexer_tc_supported(a))
+  if (indexer_runs_tc(d, a))
     return launch_indexer_tc(a, at(ws, p.indexer), p.indexer_bytes, s);
   return launch_indexer_simt(a, s);
 }
@@ -609,6 +613,8 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   ia.hist = fused_hist(dims, ia, ws, p);
   if (ia.hist && (st = ws_hist_ready(ws, p, s))) return st;
   ws_zero_forget(ws);
+  // a cluster top-k follows: the indexer lets it launch only at its end
+  ia.late_trigger = indexer_runs_tc(dims, ia) && topk_uses_clusters(rows->num_rows);
   stage_event(0, s);
   if ((st = run_indexer(dims, ia, ws, p, s))) return st;
   stage_event(1, s);
@@ -622,6 +628,7 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   ta.status = reinterpret_cast<DeviceStatus*>(ws);
   ta.trace = trace_buffer() ? trace_buffer() + kTraceTopk : nullptr;
   ta.hist = ia.hist;
+  ta.after_late_trigger = ia.late_trigger;
   if ((st = launch_topk(ta, rows->max_klen, s))) return st;
   stage_event(2, s);
   MlaArgs ma = mla_args(dims, rows, cache, q, idx, out, lse, ws, p);
@@ -675,6 +682,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     if (ia.hist && !used_hist && (st = ws_hist_ready(ws, p, s))) return st;
     if (r0 == 0) ws_zero_forget(ws);
     used_hist = used_hist || ia.hist != nullptr;
+    ia.late_trigger = indexer_runs_tc(dims, ia) && topk_uses_clusters(n);
     if ((st = run_indexer(dims, ia, ws, p, s))) return st;
     TopkArgs ta{};
     ta.num_rows = n;
@@ -686,6 +694,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     ta.status = reinterpret_cast<DeviceStatus*>(ws);
     ta.trace = trace_buffer() ? trace_buffer() + kTraceTopk : nullptr;
     ta.hist = ia.hist;
+    ta.after_late_trigger = ia.late_trigger;
     if ((st = launch_topk(ta, rows->max_klen, s))) return st;
     MlaArgs ma = mla_args(dims, &cr, cache, qq, idx, oo, ll, ws, p);
     if ((st = run_mla(dims, ma, s))) return st;

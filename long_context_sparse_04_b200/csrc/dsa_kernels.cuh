@@ -25,6 +25,8 @@ struct IndexerArgs {
   DeviceStatus* status;
   int32_t* tile_offsets;      // workspace: [n_groups + 1] exclusive scan of key tiles
   uint32_t* hist;             // [num_rows, 4096] score-key histograms (zeroed), or null
+  int late_trigger;           // tensor-core kernel: let dependents launch only once a CTA's
+                              // tiles are done (the next kernel is a cluster top-k)
 };
 
 struct TopkArgs {
@@ -38,6 +40,7 @@ struct TopkArgs {
   long long* trace;           // profiling stamps or null
   uint32_t* hist;             // [T, 4096] histograms of the scores' top 12 key bits from the
                               // indexer (read, then zeroed), or null: top-k builds its own
+  int after_late_trigger;     // the previous kernel lets dependents launch at its end only
 };
 
 struct MlaArgs {
@@ -110,6 +113,8 @@ dsa_status launch_mla_simt(const MlaArgs& a, cudaStream_t stream);
 dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream);
 bool mla_tc_supported(const MlaArgs& a);
 int mla_tc_splits(int num_rows);
+// Whether a top-k of `num_rows` rows runs as clusters (else one CTA per row).
+bool topk_uses_clusters(int num_rows);
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
 
 dsa_status launch_cache_append(const AppendArgs& a, cudaStream_t stream);

@@ -121,6 +121,7 @@ struct TcArgs {
   int64_t ld;
   uint32_t* hist;             // [num_rows, 4096] score-key histograms to add to, or null
   DeviceStatus* status;
+  int late_trigger;           // dependents launch once every CTA's tiles are done
 };
 
 // Walks the flattened (group, key tile) list from a start tile.
@@ -191,7 +192,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lim = a.spin_limit;
-  pdl_launch_dependents();
+  // dependents may launch now, or (late_trigger) once this CTA's tiles are done
+  if (!a.late_trigger) pdl_launch_dependents();
   pdl_wait();
   trace_kernel(a.status, DSA_KERNEL_INDEXER_TC);
 
@@ -507,6 +509,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       for (int k = 0; k < NSET; ++k) it.next();
     }
   }
+  if (a.late_trigger) pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -574,6 +577,7 @@ dsa_status launch_nq(const IndexerArgs& a, cudaStream_t stream) {
     t.ld = a.ld_scores;
     t.hist = a.hist ? a.hist + (int64_t)r0 * kHistBins : nullptr;
     t.status = a.status;
+    t.late_trigger = a.late_trigger;
     t.trace = trace_buffer() ? trace_buffer() + kTraceIdx : nullptr;
     t.spin_limit = fault_spin_limit();
     t.inject = fault_inject();

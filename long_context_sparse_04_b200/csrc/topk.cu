@@ -960,6 +960,10 @@ int max_topk_clusters(const void* fn, int which, int csize, size_t smem) {
   return n;
 }
 
+// Many rows (a prefill chunk) fill the device with one CTA per row; a few
+// long rows (decode) keep each row's scores in the shared memory of a cluster.
+bool topk_uses_clusters(int num_rows) { return num_rows < 2 * device_sm_count(); }
+
 // The row kernel: one CTA per row, streaming the scores.
 dsa_status launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(RowSmem);
@@ -988,9 +992,7 @@ dsa_status launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
 
 dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
-  // Many rows (a prefill chunk) fill the device with one CTA per row; a few
-  // long rows (decode) keep each row's scores in the shared memory of a cluster.
-  if (a.num_rows >= 2 * device_sm_count()) return launch_topk_rows(a, stream);
+  if (!topk_uses_clusters(a.num_rows)) return launch_topk_rows(a, stream);
   int csize = 1;
   while (csize < kMaxCluster && (int64_t)csize * kCacheCap < (int64_t)max_klen) csize <<= 1;
   const size_t smem = sizeof(TopkSmem);
@@ -1014,10 +1016,12 @@ dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   // A programmatic launch places the clusters while the previous kernel's last
   // CTAs still hold SMs; clusters of four or more CTAs placed piecemeal pack
   // worse, and a grid that fits the device in one wave of clusters may then
-  // need two.  Such a grid is launched once the previous kernel is done.
+  // need two.  Such a grid is launched once the previous kernel is done,
+  // unless that kernel lets its dependents launch only at its end (the
+  // indexer of this library's fused calls does).
   const bool one_wave =
       csize >= 4 && a.num_rows <= max_topk_clusters(fn, a.hist ? 1 : 0, csize, smem);
-  cfg.numAttrs = one_wave ? 1 : 2;
+  cfg.numAttrs = (one_wave && !a.after_late_trigger) ? 1 : 2;
   cudaError_t e = a.hist ? cudaLaunchKernelEx(&cfg, topk_kernel<true>, a)
                          : cudaLaunchKernelEx(&cfg, topk_kernel<false>, a);
   if (e != cudaSuccess) {
