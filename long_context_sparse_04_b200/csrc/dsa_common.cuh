@@ -214,6 +214,14 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
 }
+// The two halves of cluster_sync(), for threads that have work to do between
+// them; every thread that arrives also waits before it arrives again.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // Address of the same smem object in CTA `rank` of the cluster (shared::cluster window).
 __device__ __forceinline__ uint32_t mapa(const void* p, uint32_t rank) {
   uint32_t r;

@@ -314,21 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   if (threadIdx.x == 0 && a.merge_in_cluster) mbar_expect_tx(&S.m_full, kMergeTx);
   const bool gather_warp = warp >= kGatherWarp0 && warp < kGatherWarp0 + kGatherWarps;
   const int g = threadIdx.x - 32 * kGatherWarp0;          // gather thread index (0..479)
-  // Q first: its pieces land while the selection is resolved below (the
-  // gather warps arrive on q_full for them once the barrier init is visible)
-  if (gather_warp && nblk > 0) {
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
-    for (int qi = g; qi < kH * kPieces; qi += kGatherThreads) {
-      const int h = qi / kPieces, c = qi - h * kPieces;
-      if (c < 32) {
-        cp_async_16(S.q[c >> 3] + sw128_off(h, c & 7), qrow + h * kD + 256 * rank + 8 * c);
-      } else {
-        cp_async_16(S.q_rope + sw64_off(h, c - 32), qrow + h * kD + kDC + 32 * rank + 8 * (c - 32));
-      }
-    }
-  }
   // physical rows of the selected keys of this split (entries past nvalid are
-  // none): all index loads of a thread first, then all its block-table loads
+  // none): the index loads go out first (they gate the first gather), then the
+  // Q pieces, then the block-table loads
   {
     constexpr int kPer = (kMaxKeys + kThreads - 1) / kThreads;
     const int32_t* idx = a.idx + (int64_t)t * a.topk + k0;
@@ -338,6 +326,19 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     for (int u = 0; u < kPer; ++u) {
       const int i = threadIdx.x + u * kThreads;
       sv[u] = i < nvalid ? __ldg(idx + i) : -1;
+    }
+    // then Q: its pieces land while the selection is resolved below (the
+    // gather warps arrive on q_full for them once the barrier init is visible)
+    if (gather_warp && nblk > 0) {
+      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t)t * kH * kD;
+      for (int qi = g; qi < kH * kPieces; qi += kGatherThreads) {
+        const int h = qi / kPieces, c = qi - h * kPieces;
+        if (c < 32) {
+          cp_async_16(S.q[c >> 3] + sw128_off(h, c & 7), qrow + h * kD + 256 * rank + 8 * c);
+        } else {
+          cp_async_16(S.q_rope + sw64_off(h, c - 32), qrow + h * kD + kDC + 32 * rank + 8 * (c - 32));
+        }
+      }
     }
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
@@ -361,7 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();   // the peer's barriers are initialised before any remote arrive
+  // Every CTA of the cluster has initialised its barriers: the exchange and
+  // softmax warpgroups, which touch other CTAs' shared memory, wait for that;
+  // the gather and MMA warpgroups, which touch only their own, start at once.
+  cluster_arrive();
   const uint32_t tmem = S.tmem_base;
   // Registers: the gather / MMA warpgroups (0-3) give theirs to the exchange
   // and softmax warpgroups (4-6).  Each warpgroup executes one setmaxnreg, at
@@ -392,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
       }
       cp_async_wait_all();
     }
+    cluster_wait();
   } else if (warp < kSmWarp0) {
     setmaxnreg_inc_high();
+    cluster_wait();
     // ------------------------------------------------------------ exchange (128 threads)
     // Copies this CTA's partial logits of block j to the peer with one bulk copy
     // while the softmax warpgroups are still working on block j-1.  A wait that
@@ -429,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_tc_kernel(MlaArgs a, int keys
     if (h == 0) bulk_wait_read0();
   } else {
     setmaxnreg_inc_high();
+    cluster_wait();
     // ------------------------------------------------------------ softmax / output (256 threads)
     // Thread (half, h): head h (= TMEM lane), keys [32 half, 32 half + 32) of
     // every block, value dims [128 half, 128 half + 128) of this CTA's 256 in
