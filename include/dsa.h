@@ -205,7 +205,8 @@ dsa_status dsa_set_stage_events(void* const* events, int32_t n_events);
  * own region: int64 [0, 512) the sparse-MLA kernel's first CTA pair
  * ([2 CTAs][8 events][32 blocks]: decoded, after the max barrier, S issued,
  * PV issued, S read by the softmax, peer logits arrived, P stored, exp done),
- * [512, 640) top-k's first cluster ([8 CTAs][16 events], phase ends), and
+ * [512, 640) top-k's first cluster ([8 CTAs][16 events], phase ends; the
+ * cluster kernel only), and
  * [640, 896) the indexer's CTA 0 ([8 events][32 tiles]: stage free, TMA
  * issued, MMA ready, MMA committed, accumulator ready, key data landed,
  * accumulator loaded, scores stored).  Stamps of one SM's clock; compare

@@ -614,7 +614,7 @@ dsa_status dsa_decode_step(const dsa_dims* dims, const dsa_rows* rows, const dsa
   if (ia.hist && (st = ws_hist_ready(ws, p, s))) return st;
   ws_zero_forget(ws);
   // a cluster top-k follows: the indexer lets it launch only at its end
-  ia.late_trigger = indexer_runs_tc(dims, ia) && topk_uses_clusters(rows->num_rows);
+  ia.late_trigger = indexer_runs_tc(dims, ia) && topk_uses_clusters(rows->num_rows, rows->max_klen);
   stage_event(0, s);
   if ((st = run_indexer(dims, ia, ws, p, s))) return st;
   stage_event(1, s);
@@ -682,7 +682,7 @@ dsa_status dsa_forward(const dsa_dims* dims, const dsa_rows* rows, const dsa_cac
     if (ia.hist && !used_hist && (st = ws_hist_ready(ws, p, s))) return st;
     if (r0 == 0) ws_zero_forget(ws);
     used_hist = used_hist || ia.hist != nullptr;
-    ia.late_trigger = indexer_runs_tc(dims, ia) && topk_uses_clusters(n);
+    ia.late_trigger = indexer_runs_tc(dims, ia) && topk_uses_clusters(n, rows->max_klen);
     if ((st = run_indexer(dims, ia, ws, p, s))) return st;
     TopkArgs ta{};
     ta.num_rows = n;

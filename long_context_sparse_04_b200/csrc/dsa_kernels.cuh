@@ -113,8 +113,9 @@ dsa_status launch_mla_simt(const MlaArgs& a, cudaStream_t stream);
 dsa_status launch_mla_tc(const MlaArgs& a, cudaStream_t stream);
 bool mla_tc_supported(const MlaArgs& a);
 int mla_tc_splits(int num_rows);
-// Whether a top-k of `num_rows` rows runs as clusters (else one CTA per row).
-bool topk_uses_clusters(int num_rows);
+// Whether a top-k of `num_rows` rows of at most `max_klen` keys runs as
+// clusters (else one CTA per row, streaming).
+bool topk_uses_clusters(int num_rows, int max_klen);
 size_t mla_ws_bytes(int num_rows, int n_heads, int d_c, int splits);
 
 dsa_status launch_cache_append(const AppendArgs& a, cudaStream_t stream);

@@ -30,8 +30,9 @@
 //    contiguous range and warp ballots giving the order inside it.
 // Rows with klen <= k return 0..klen-1 then -1.
 //
-// Batches of at least two rows per SM (prefill chunks) run topk_row_kernel
-// instead (further below): one CTA per row streaming the scores, no cluster.
+// Batches of at least two rows per SM longer than one CTA's cache (long
+// prefill chunks) run topk_row_kernel instead (further below): one CTA per
+// row streaming the scores, no cluster.
 #include "dsa_kernels.cuh"
 
 namespace dsa {
@@ -960,9 +961,13 @@ int max_topk_clusters(const void* fn, int which, int csize, size_t smem) {
   return n;
 }
 
-// Many rows (a prefill chunk) fill the device with one CTA per row; a few
-// long rows (decode) keep each row's scores in the shared memory of a cluster.
-bool topk_uses_clusters(int num_rows) { return num_rows < 2 * device_sm_count(); }
+// Many long rows (a prefill chunk past 16K keys) fill the device with one CTA
+// per row; a few long rows (decode) keep each row's scores in the shared
+// memory of a cluster, and rows that fit one CTA's cache take one CTA with the
+// row in shared memory.
+bool topk_uses_clusters(int num_rows, int max_klen) {
+  return num_rows < 2 * device_sm_count() || max_klen <= kCacheCap;
+}
 
 // The row kernel: one CTA per row, streaming the scores.
 dsa_status launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
@@ -992,7 +997,7 @@ dsa_status launch_topk_rows(const TopkArgs& a, cudaStream_t stream) {
 
 dsa_status launch_topk(const TopkArgs& a, int max_klen, cudaStream_t stream) {
   if (a.num_rows == 0) return DSA_OK;
-  if (!topk_uses_clusters(a.num_rows)) return launch_topk_rows(a, stream);
+  if (!topk_uses_clusters(a.num_rows, max_klen)) return launch_topk_rows(a, stream);
   int csize = 1;
   while (csize < kMaxCluster && (int64_t)csize * kCacheCap < (int64_t)max_klen) csize <<= 1;
   const size_t smem = sizeof(TopkSmem);

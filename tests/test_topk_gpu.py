@@ -121,11 +121,12 @@ def test_topk_rows_beyond_the_cluster_cache(N, kind):
 
 @pytest.mark.parametrize("k", [2048, 64])
 def test_topk_many_rows(N, k):
-    """A batch of hundreds of rows runs one CTA per row, streaming the scores
-    (the cluster kernel above runs the few-row batches): every kind of row,
+    """A batch of hundreds of rows, some past one CTA's cache, runs one CTA
+    per row streaming the scores (the cluster kernel above runs the few-row
+    batches and batches of short rows): every kind of row,
     lengths around k and well past it, and bins far over the threshold-bin
     capacity (all_equal, crowded_bin), each against the oracle."""
-    lengths = [1, k - 1, k, k + 1, 3000, 4097, 6000, 9000, 20000]
+    lengths = [1, k - 1, k, k + 1, 3000, 4097, 6000, 9000, 20000, 40000]
     import torch
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     rows = []
