@@ -18,7 +18,12 @@
 // derivative is 1 where its argument is > 0, else 0.  The argument's sign is
 // taken exactly: q_j . k_s = q_scale_j k_scale_s sum_i e4m3(q8_ji) e4m3(k8_si),
 // and that sum of products of E4M3 values (each a multiple of 2^-9 below 449)
-// is exact in fp64, so the mask does not depend on summation order.
+// is exact in fp64, so the mask does not depend on summation order.  The dot
+// products run in fp32 first: a sum of 128 terms accumulated with fma is
+// within gamma_127 sum_i |k_i q_i| <= gamma_127 |k| |q| of exact
+// (gamma_n = n u / (1 - n u), u = 2^-24; Cauchy-Schwarz for the second step),
+// so its sign is the exact sign whenever its magnitude exceeds that bound; the
+// few that do not are recomputed in fp64.
 // Every sum is in a fixed order: results are deterministic run to run.
 #include <cuda_fp8.h>
 
@@ -31,14 +36,37 @@ constexpr int kHI = 64, kDI = 128;        // the shapes these kernels run (H_I x
 constexpr int kTile = 32;                 // keys per inner tile
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ float e4m3_to_float(uint8_t c) {
-  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
-  return __half2float(__half(h));
+// Sixteen e4m3 codes (one 16-byte piece) as floats.
+__device__ __forceinline__ void e4m3x16_to_float(uint4 v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+      const float2 x = __half22float2(__half2(r));
+      f[4 * i + 2 * h] = x.x;
+      f[4 * i + 2 * h + 1] = x.y;
+    }
+  }
 }
-// Stored value of element i of an indexer tensor (e4m3 code or f32), unscaled.
-__device__ __forceinline__ float idx_elem(const void* p, int64_t i, bool fp8) {
-  return fp8 ? e4m3_to_float(static_cast<const uint8_t*>(p)[i]) : static_cast<const float*>(p)[i];
+// Elements [16 p, 16 p + 16) of an indexer tensor row block (e4m3 codes or
+// f32), unscaled, as floats; `base` is 16-byte aligned.
+__device__ __forceinline__ void load16(const void* base, int64_t p, bool fp8, float* f) {
+  if (fp8) {
+    e4m3x16_to_float(reinterpret_cast<const uint4*>(base)[p], f);
+  } else {
+    const float4* b = reinterpret_cast<const float4*>(base) + 4 * p;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = b[i];
+      f[4 * i] = x.x; f[4 * i + 1] = x.y; f[4 * i + 2] = x.z; f[4 * i + 3] = x.w;
+    }
+  }
 }
+// fp32 filter factor: gamma_127 for u = 2^-24, rounded up with some room.
+constexpr double kDotBound = 7.6e-6;
 
 __device__ __forceinline__ float block_reduce_sum(float v, float* tmp) {
 #pragma unroll
@@ -90,10 +118,11 @@ __global__ void __launch_bounds__(kThreads) indexer_kl_kernel(WarmupArgs a) {
   if (threadIdx.x == 0) a.loss[t] = n > 0 ? kl : 0.f;
 }
 
-// One key tile: stored key values (unscaled) and their scales into shared
-// memory; keys past klen or unmapped read as zero with scale 0.
+// One key tile: stored key values (unscaled), their scales and the fp32
+// filter bound factor kDotBound |k_s| into shared memory; keys past klen or
+// unmapped read as zero with scale 0.
 __device__ __forceinline__ void load_key_tile(const WarmupArgs& a, int seq, int s0, int klen,
-                                              float (*kv)[kDI], float* ks, int64_t* prow) {
+                                              float (*kv)[kDI], float* ks, float* kn, int64_t* prow) {
   const bool fp8 = a.idx_dtype == DSA_FP8_E4M3;
   if (threadIdx.x < kTile) {
     const int s = s0 + threadIdx.x;
@@ -107,20 +136,51 @@ __device__ __forceinline__ void load_key_tile(const WarmupArgs& a, int seq, int 
     ks[threadIdx.x] = r >= 0 ? (a.idx_k_scale ? a.idx_k_scale[r] : 1.f) : 0.f;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kTile * kDI; i += kThreads) {
-    const int j = i / kDI, d = i - j * kDI;
+  // 32 keys x 8 pieces of 16 elements: one piece per thread
+  {
+    const int j = threadIdx.x >> 3, pc = threadIdx.x & 7;
     const int64_t r = prow[j];
-    kv[j][d] = r >= 0 ? idx_elem(a.idx_k, r * kDI + d, fp8) : 0.f;
+    float f[16];
+    if (r >= 0) {
+      load16(static_cast<const uint8_t*>(a.idx_k) + r * kDI * (fp8 ? 1 : 4), pc, fp8, f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) f[e] = 0.f;
+    }
+    double ss = 0.0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ss = fma((double)f[e], (double)f[e], ss);
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) *reinterpret_cast<float4*>(&kv[j][16 * pc + e]) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+    // |k_s|^2 over the eight pieces of the key (lanes 8j'..8j'+7 of a warp)
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (pc == 0) kn[j] = (float)(kDotBound * sqrt(ss) * (1.0 + 1e-6));
   }
   __syncthreads();
 }
 
-// The query of row t: stored values (unscaled), scales, weights.
+// The query of row t: stored values (unscaled), scales, weights, and |q_j|.
 __device__ __forceinline__ void load_query(const WarmupArgs& a, int t, float (*qv)[kDI], float* qs,
-                                           float* w) {
+                                           float* w, float* qn) {
   const bool fp8 = a.idx_dtype == DSA_FP8_E4M3;
-  for (int i = threadIdx.x; i < kHI * kDI; i += kThreads)
-    qv[i / kDI][i % kDI] = idx_elem(a.q_idx, (int64_t)t * kHI * kDI + i, fp8);
+  const uint8_t* base = static_cast<const uint8_t*>(a.q_idx) + (int64_t)t * kHI * kDI * (fp8 ? 1 : 4);
+  // 64 heads x 8 pieces of 16 elements: two pieces per thread
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const int piece = threadIdx.x + kThreads * h2;
+    const int j = piece >> 3, pc = piece & 7;
+    float f[16];
+    load16(base + (int64_t)j * kDI * (fp8 ? 1 : 4), pc, fp8, f);
+    double ss = 0.0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ss = fma((double)f[e], (double)f[e], ss);
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) *reinterpret_cast<float4*>(&qv[j][16 * pc + e]) = make_float4(f[e], f[e + 1], f[e + 2], f[e + 3]);
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (pc == 0) qn[j] = (float)(sqrt(ss) * (1.0 + 1e-6));
+  }
   if (threadIdx.x < kHI) {
     qs[threadIdx.x] = a.q_scale ? a.q_scale[(int64_t)t * kHI + threadIdx.x] : 1.f;
     w[threadIdx.x] = a.w[(int64_t)t * kHI + threadIdx.x];
@@ -128,30 +188,43 @@ __device__ __forceinline__ void load_query(const WarmupArgs& a, int t, float (*q
   __syncthreads();
 }
 
-// dots[s][j] = sum_i kv[s][i] qv[j][i] in fp64 (exact for e4m3 values), for
-// the 32 x 64 (key, head) pairs of a tile.  Thread tid takes keys ks, ks + 16
-// (ks = tid / 16) and heads jh + 16c (jh = tid % 16, c < 4): 6 shared loads per
-// 8 FMAs.  Each thread walks the dims from its own start 2 jh + ks, so the 32
-// lanes of a warp read 32 different banks.
-__device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kDI], double (*dots)[kHI]) {
+// dots[s][j] = sum_i kv[s][i] qv[j][i] for the 32 x 64 (key, head) pairs of a
+// tile, with its sign exact: fp32 fma sums, and the pairs within the bound
+// kn[s] qn[j] of zero recomputed in fp64 (exact for e4m3 values).  A nonzero
+// exact value keeps its sign in the stored float.  Thread tid takes keys ks,
+// ks + 16 (ks = tid / 16) and heads jh + 16c (jh = tid % 16, c < 4): 6 shared
+// loads per 8 FMAs.  Each thread walks the dims from its own start 2 jh + ks,
+// so the 32 lanes of a warp read 32 different banks.
+__device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kDI], const float* kn,
+                                          const float* qn, float (*dots)[kHI]) {
   const int ks = threadIdx.x >> 4, jh = threadIdx.x & 15;
   const int rot = 2 * jh + ks;
-  double acc[2][4] = {{0.0, 0.0, 0.0, 0.0}, {0.0, 0.0, 0.0, 0.0}};
-#pragma unroll 4
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
   for (int i = 0; i < kDI; ++i) {
     const int ii = (i + rot) & (kDI - 1);
-    const double k0 = kv[ks][ii], k1 = kv[ks + 16][ii];
+    const float k0 = kv[ks][ii], k1 = kv[ks + 16][ii];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const double q = qv[jh + 16 * c][ii];
-      acc[0][c] = fma(k0, q, acc[0][c]);
-      acc[1][c] = fma(k1, q, acc[1][c]);
+      const float q = qv[jh + 16 * c][ii];
+      acc[0][c] = fmaf(k0, q, acc[0][c]);
+      acc[1][c] = fmaf(k1, q, acc[1][c]);
     }
   }
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    dots[ks][jh + 16 * c] = acc[0][c];
-    dots[ks + 16][jh + 16 * c] = acc[1][c];
+  for (int r = 0; r < 2; ++r) {
+    const int s = ks + 16 * r;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = jh + 16 * c;
+      float d = acc[r][c];
+      if (fabsf(d) <= kn[s] * qn[j]) {             // the sign is not certain: exact sum
+        double e = 0.0;
+        for (int i = 0; i < kDI; ++i) e = fma((double)kv[s][i], (double)qv[j][i], e);
+        d = e > 0.0 ? fmaxf((float)e, 1e-45f) : (e < 0.0 ? fminf((float)e, -1e-45f) : 0.f);
+      }
+      dots[s][j] = d;
+    }
   }
   __syncthreads();
 }
@@ -159,14 +232,16 @@ __device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kDI], do
 struct DqSmem {
   float qv[kHI][kDI];
   float kv[kTile][kDI];
-  double dots[kTile][kHI];
+  float dots[kTile][kHI];
   float coef[kTile][kHI];                  // g_s w_j [dot > 0] k_scale_s
-  float qs[kHI], w[kHI], ks[kTile], g[kTile];
+  float qs[kHI], w[kHI], ks[kTile], g[kTile], kn[kTile], qn[kHI];
   int64_t prow[kTile];
 };
 
 // grid (n_chunks, T), block 256.  Thread tid accumulates dq[j][d] for
-// j = tid / 4 (heads 0..63) and d = tid % 4 + 4i (i < 32), and (tid < 64) dw[tid].
+// j = tid / 4 (heads 0..63) and d = 16 i + 4 (tid % 4) + e (i < 8, e < 4: four
+// dims per 16-byte load; the four threads of a head read 64 contiguous bytes),
+// and (tid < 64) dw[tid].
 __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   DqSmem& S = *reinterpret_cast<DqSmem*>(smraw);
@@ -174,32 +249,38 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) 
   const int t = blockIdx.y, c = blockIdx.x;
   const int klen = a.row_klen[t], seq = a.row_seq[t];
   const int s_lo = c * a.chunk_keys, s_hi = min(klen, s_lo + a.chunk_keys);
-  const int jq = threadIdx.x >> 2, d0 = threadIdx.x & 3;
+  const int jq = threadIdx.x >> 2, d0 = 4 * (threadIdx.x & 3);
   float acc[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) acc[i] = 0.f;
   float dw = 0.f;
   if (s_lo < s_hi) {
-    load_query(a, t, S.qv, S.qs, S.w);
+    load_query(a, t, S.qv, S.qs, S.w, S.qn);
     const float* g = a.grad + (int64_t)t * a.ld_grad;
     for (int s0 = s_lo; s0 < s_hi; s0 += kTile) {
-      load_key_tile(a, seq, s0, s_hi, S.kv, S.ks, S.prow);
+      load_key_tile(a, seq, s0, s_hi, S.kv, S.ks, S.kn, S.prow);
       if (threadIdx.x < kTile) S.g[threadIdx.x] = s0 + threadIdx.x < s_hi ? g[s0 + threadIdx.x] : 0.f;
-      tile_dots(S.kv, S.qv, S.dots);
+      tile_dots(S.kv, S.qv, S.kn, S.qn, S.dots);
       for (int e = threadIdx.x; e < kTile * kHI; e += kThreads) {
         const int s = e / kHI, j = e - s * kHI;
-        S.coef[s][j] = S.dots[s][j] > 0.0 ? S.g[s] * S.w[j] * S.ks[s] : 0.f;
+        S.coef[s][j] = S.dots[s][j] > 0.f ? S.g[s] * S.w[j] * S.ks[s] : 0.f;
       }
       __syncthreads();
       if (threadIdx.x < kHI) {                        // dw_j += sum_s g_s ReLU(q_j . k_s)
         const int j = threadIdx.x;
         for (int s = 0; s < kTile; ++s)
-          dw = fmaf(S.g[s] * S.ks[s] * S.qs[j], (float)fmax(S.dots[s][j], 0.0), dw);
+          dw = fmaf(S.g[s] * S.ks[s] * S.qs[j], fmaxf(S.dots[s][j], 0.f), dw);
       }
       for (int s = 0; s < kTile; ++s) {               // dq_j += sum_s coef_sj k_s
         const float cf = S.coef[s][jq];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = fmaf(cf, S.kv[s][d0 + 4 * i], acc[i]);
+        for (int i = 0; i < 8; ++i) {
+          const float4 k4 = *reinterpret_cast<const float4*>(&S.kv[s][16 * i + d0]);
+          acc[4 * i] = fmaf(cf, k4.x, acc[4 * i]);
+          acc[4 * i + 1] = fmaf(cf, k4.y, acc[4 * i + 1]);
+          acc[4 * i + 2] = fmaf(cf, k4.z, acc[4 * i + 2]);
+          acc[4 * i + 3] = fmaf(cf, k4.w, acc[4 * i + 3]);
+        }
       }
       __syncthreads();
     }
@@ -207,7 +288,7 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dq_kernel(WarmupArgs a) 
   // partials [T][n_chunks][64][128 + 1]: dq then dw at column 128
   float* part = a.partial + (((int64_t)t * a.n_chunks + c) * kHI) * (kDI + 1);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) part[(int64_t)jq * (kDI + 1) + d0 + 4 * i] = acc[i];
+  for (int i = 0; i < 32; ++i) part[(int64_t)jq * (kDI + 1) + 16 * (i >> 2) + d0 + (i & 3)] = acc[i];
   if (threadIdx.x < kHI) part[(int64_t)threadIdx.x * (kDI + 1) + kDI] = dw;
 }
 
@@ -227,22 +308,23 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_reduce_kernel(WarmupArgs
 struct DkSmem {
   float qv[kHI][kDI];
   float kv[kTile][kDI];
-  double dots[kTile][kHI];
+  float dots[kTile][kHI];
   float coef[kTile][kHI];                  // g_s w_j [dot > 0] q_scale_j
-  float qs[kHI], w[kHI], ks[kTile], g[kTile];
+  float qs[kHI], w[kHI], ks[kTile], g[kTile], kn[kTile], qn[kHI];
   int64_t prow[kTile];
   int seen[kTile];
 };
 
 // grid (ceil(max_klen / 32), num_seqs), block 256.  Thread tid accumulates
-// dk[s][d] for s = tid / 8 and d = tid % 8 + 8i (i < 16), over the rows of
-// sequence b that see key s, in row order; writes the keys some row sees.
+// dk[s][d] for s = tid / 8 and d = 32 i + 4 (tid % 8) + e (i < 4, e < 4), over
+// the rows of sequence b that see key s, in row order; writes the keys some
+// row sees.
 __global__ void __launch_bounds__(kThreads) indexer_bwd_dk_kernel(WarmupArgs a) {
   extern __shared__ __align__(16) uint8_t smraw[];
   DkSmem& S = *reinterpret_cast<DkSmem*>(smraw);
   trace_kernel(a.status, DSA_KERNEL_WARMUP);
   const int b = blockIdx.y, s0 = blockIdx.x * kTile;
-  const int sk = threadIdx.x >> 3, d0 = threadIdx.x & 7;
+  const int sk = threadIdx.x >> 3, d0 = 4 * (threadIdx.x & 7);
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
@@ -259,35 +341,42 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_dk_kernel(WarmupArgs a) 
   kmax = 0;
   for (int i = 0; i < kThreads / 32; ++i) kmax = max(kmax, kmax_w[i]);
   if (s0 >= kmax) return;                            // no row of b sees this tile
-  load_key_tile(a, b, s0, kmax, S.kv, S.ks, S.prow);
+  load_key_tile(a, b, s0, kmax, S.kv, S.ks, S.kn, S.prow);
   for (int t = 0; t < a.num_rows; ++t) {
     if (a.row_seq[t] != b) continue;                  // uniform over the block
     const int klen = a.row_klen[t];
     if (klen <= s0) continue;
-    load_query(a, t, S.qv, S.qs, S.w);
+    load_query(a, t, S.qv, S.qs, S.w, S.qn);
     const float* g = a.grad + (int64_t)t * a.ld_grad;
     if (threadIdx.x < kTile) {
       const bool vis = s0 + threadIdx.x < klen;
       S.g[threadIdx.x] = vis ? g[s0 + threadIdx.x] : 0.f;
       S.seen[threadIdx.x] |= vis ? 1 : 0;
     }
-    tile_dots(S.kv, S.qv, S.dots);
+    tile_dots(S.kv, S.qv, S.kn, S.qn, S.dots);
     for (int e = threadIdx.x; e < kTile * kHI; e += kThreads) {
       const int s = e / kHI, j = e - s * kHI;
-      S.coef[s][j] = S.dots[s][j] > 0.0 ? S.g[s] * S.w[j] * S.qs[j] : 0.f;
+      S.coef[s][j] = S.dots[s][j] > 0.f ? S.g[s] * S.w[j] * S.qs[j] : 0.f;
     }
     __syncthreads();
     for (int j = 0; j < kHI; ++j) {                   // dk_s += sum_j coef_sj q_j
       const float cf = S.coef[sk][j];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = fmaf(cf, S.qv[j][d0 + 8 * i], acc[i]);
+      for (int i = 0; i < 4; ++i) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&S.qv[j][32 * i + d0]);
+        acc[4 * i] = fmaf(cf, q4.x, acc[4 * i]);
+        acc[4 * i + 1] = fmaf(cf, q4.y, acc[4 * i + 1]);
+        acc[4 * i + 2] = fmaf(cf, q4.z, acc[4 * i + 2]);
+        acc[4 * i + 3] = fmaf(cf, q4.w, acc[4 * i + 3]);
+      }
     }
     __syncthreads();
   }
   if (S.seen[sk] && S.prow[sk] >= 0) {
     float* dst = a.dk + S.prow[sk] * kDI + d0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) dst[8 * i] = acc[i];
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(dst + 32 * i) = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
   }
 }
 
