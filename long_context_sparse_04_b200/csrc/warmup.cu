@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kHI = 64, kDI = 128;        // the shapes these kernels run (H_I x d_I)
 constexpr int kTile = 32;                 // keys per inner tile
+constexpr int kQP = kDI + 4;              // padded row of a query in shared memory
 constexpr int kThreads = 256;
 
 // Sixteen e4m3 codes (one 16-byte piece) as floats.
@@ -161,7 +162,7 @@ __device__ __forceinline__ void load_key_tile(const WarmupArgs& a, int seq, int 
 }
 
 // The query of row t: stored values (unscaled), scales, weights, and |q_j|.
-__device__ __forceinline__ void load_query(const WarmupArgs& a, int t, float (*qv)[kDI], float* qs,
+__device__ __forceinline__ void load_query(const WarmupArgs& a, int t, float (*qv)[kQP], float* qs,
                                            float* w, float* qn) {
   const bool fp8 = a.idx_dtype == DSA_FP8_E4M3;
   const uint8_t* base = static_cast<const uint8_t*>(a.q_idx) + (int64_t)t * kHI * kDI * (fp8 ? 1 : 4);
@@ -191,32 +192,34 @@ __device__ __forceinline__ void load_query(const WarmupArgs& a, int t, float (*q
 // dots[s][j] = sum_i kv[s][i] qv[j][i] for the 32 x 64 (key, head) pairs of a
 // tile, with its sign exact: fp32 fma sums, and the pairs within the bound
 // kn[s] qn[j] of zero recomputed in fp64 (exact for e4m3 values).  A nonzero
-// exact value keeps its sign in the stored float.  Thread tid takes keys ks,
-// ks + 16 (ks = tid / 16) and heads jh + 16c (jh = tid % 16, c < 4): 6 shared
-// loads per 8 FMAs.  Each thread walks the dims from its own start 2 jh + ks,
-// so the 32 lanes of a warp read 32 different banks.
-__device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kDI], const float* kn,
+// exact value keeps its sign in the stored float.  Thread (warp w, lane l)
+// takes keys 4w .. 4w + 3 and heads l, l + 32: per four dims, each key's
+// values are one 16-byte load that the warp shares, each head's one 16-byte
+// load (query rows padded to kQP floats, so the 8 lanes of a quarter warp hit
+// distinct banks): 6 loads per 32 FMAs.
+__device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kQP], const float* kn,
                                           const float* qn, float (*dots)[kHI]) {
-  const int ks = threadIdx.x >> 4, jh = threadIdx.x & 15;
-  const int rot = 2 * jh + ks;
-  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 8
-  for (int i = 0; i < kDI; ++i) {
-    const int ii = (i + rot) & (kDI - 1);
-    const float k0 = kv[ks][ii], k1 = kv[ks + 16][ii];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float acc[4][2];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float q = qv[jh + 16 * c][ii];
-      acc[0][c] = fmaf(k0, q, acc[0][c]);
-      acc[1][c] = fmaf(k1, q, acc[1][c]);
+  for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < kDI; i += 4) {
+    const float4 q0 = *reinterpret_cast<const float4*>(&qv[lane][i]);
+    const float4 q1 = *reinterpret_cast<const float4*>(&qv[lane + 32][i]);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 k = *reinterpret_cast<const float4*>(&kv[4 * w + r][i]);
+      acc[r][0] = fmaf(k.w, q0.w, fmaf(k.z, q0.z, fmaf(k.y, q0.y, fmaf(k.x, q0.x, acc[r][0]))));
+      acc[r][1] = fmaf(k.w, q1.w, fmaf(k.z, q1.z, fmaf(k.y, q1.y, fmaf(k.x, q1.x, acc[r][1]))));
     }
   }
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int s = ks + 16 * r;
+  for (int r = 0; r < 4; ++r) {
+    const int s = 4 * w + r;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = jh + 16 * c;
+    for (int c = 0; c < 2; ++c) {
+      const int j = lane + 32 * c;
       float d = acc[r][c];
       if (fabsf(d) <= kn[s] * qn[j]) {             // the sign is not certain: exact sum
         double e = 0.0;
@@ -230,7 +233,7 @@ __device__ __forceinline__ void tile_dots(float (*kv)[kDI], float (*qv)[kDI], co
 }
 
 struct DqSmem {
-  float qv[kHI][kDI];
+  float qv[kHI][kQP];
   float kv[kTile][kDI];
   float dots[kTile][kHI];
   float coef[kTile][kHI];                  // g_s w_j [dot > 0] k_scale_s
@@ -306,7 +309,7 @@ __global__ void __launch_bounds__(kThreads) indexer_bwd_reduce_kernel(WarmupArgs
 }
 
 struct DkSmem {
-  float qv[kHI][kDI];
+  float qv[kHI][kQP];
   float kv[kTile][kDI];
   float dots[kTile][kHI];
   float coef[kTile][kHI];                  // g_s w_j [dot > 0] q_scale_j
