@@ -167,7 +167,9 @@ size_t dsa_workspace_size(const dsa_dims* dims, const dsa_rows* rows, dsa_op op)
  * short may leave histograms behind).  A workspace may then serve calls of
  * other ops or other rows in any order: the library records, per workspace
  * address on the host, which bytes its calls left zeroed, and a call whose
- * histogram region is not among them clears it first (one memset). */
+ * histogram region is not among them clears it first (one memset).  A fused
+ * call on a workspace never initialised may select wrongly (its histograms
+ * hold other counts) but accesses nothing out of bounds. */
 dsa_status dsa_workspace_init(void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /* Synchronise `stream`, copy the device status word of `ws` to *status_out

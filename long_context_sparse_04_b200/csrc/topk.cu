@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
       for (int i = tid; i < kBins0 / 4; i += kThreads)
         reinterpret_cast<uint4*>(ghist)[i] = make_uint4(0u, 0u, 0u, 0u);
     for (uint32_t r = 0; r < rank; ++r) goff_h += S.cnt_b0[r];
+
   }
   kstamp(a.trace, csize, rank, 4);
 
@@ -414,6 +415,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkArgs a) {
     }
     auto send = [&](uint32_t key) {
       const uint32_t slot = goff + atomicAdd(&S.gcount, 1u);
+      // only a row histogram that does not count this row's scores (a workspace
+      // used before dsa_workspace_init) can overfill the list
+      if (slot >= (uint32_t)kGatherCap) return;
       for (uint32_t r = 0; r < csize; ++r) {
         if (r == rank) S.gather[slot] = key;
         else st_dsmem_u32(mapa(&S.gather[slot], r), key);
@@ -789,8 +793,10 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(TopkArgs a) {
               base = __shfl_sync(0xffffffffu, base, 0);
               if (mine) {
                 const uint32_t slot = base + __popc(bl & lt);
-                S.gather[slot] = key;
-                S.gwarp[slot] = (uint8_t)warp;
+                if (slot < (uint32_t)kRowGatherCap) {   // always, with consistent counts
+                  S.gather[slot] = key;
+                  S.gwarp[slot] = (uint8_t)warp;
+                }
               }
             }
           }
@@ -802,6 +808,9 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row_kernel(TopkArgs a) {
   }
   for (int i = tid; i < 2 * kBins; i += kRowThreads) (&S.lhist[0][0])[i] = 0u;
   __syncthreads();
+  // the histogram must count exactly the keys of bin B0 (a workspace used
+  // before dsa_workspace_init can hold other counts)
+  if (kHist && gathered && tid == 0 && S.gcount != c0) set_status(a.status, DSA_ERR_WORKSPACE, t);
 
   // ---- 3. T and `need`; per warp, keys of B0 above T and equal to it
   uint32_t T, need;
