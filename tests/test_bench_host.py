@@ -41,3 +41,22 @@ def test_path_stage_units():
     sel = np.minimum(klen, 2048)
     assert mla["bytes"] == int(sel.sum()) * 1152 + len(klen) * 128 * (576 + 512) * 2
     assert mla["flops"] == int(sel.sum()) * 2 * 128 * (576 + 512)
+
+
+def test_warmup_flops():
+    cfg = I.CONFIGS["decode_16k"].replace(ctx_lo=300, ctx_hi=700, n_seqs=3)
+    inp = I.generate(cfg, with_q=False, threads=2)
+    fl = bench.warmup_flops(inp)
+    pairs = int(inp["row_klen"].astype(np.int64).sum())
+    # the 64 x 128 dot products twice (dq/dw, dk) and the dq and dk contractions
+    assert fl == {"fp32": 4 * 2 * 64 * 128 * pairs, "pairs": pairs}
+
+
+def test_path_launches():
+    import types
+    n = types.SimpleNamespace(DSA_KERNEL_MLA_COMBINE=0x20)
+    # decode: indexer, top-k, attention (the split merge runs inside the attention kernel)
+    assert bench.path_launches(n, 0x20 | 0x10, 32, prefill=False) == 3
+    # prefill: the three kernels per 512-row chunk
+    assert bench.path_launches(n, 0, 65536, prefill=True) == 3 * 128
+    assert bench.path_launches(n, 0, 513, prefill=True) == 6
